@@ -1,0 +1,20 @@
+"""B200-native forward pass of one Mixture-of-Experts layer.
+
+Route (x @ W_gate, softmax, top-k, renormalise) -> permute by expert id ->
+grouped expert FFN (tcgen05 / TMEM GEMMs) -> deterministic combine, all in
+hand-written sm_100a kernels behind a C ABI (``include/moe_b200.h``).
+
+The ops live in :mod:`routing_grouped_expert_moe_b200.binding`; importing them
+loads ``lib/libmoe_b200.so`` and raises if it has not been built.
+"""
+__all__ = ["binding", "synth"]
+
+
+def __getattr__(name):
+    if name == "binding":
+        from . import binding
+        return binding
+    if name == "synth":
+        from . import synth
+        return synth
+    raise AttributeError(name)

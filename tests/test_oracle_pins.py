@@ -1,0 +1,315 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test ties one oracle function to brute force, a closed form, a library
+routine on a special case, or a hand-derived fixture under tests/golden/, so
+that a dropped term, a wrong sign or index, or a transposed operand fails.
+"""
+import json
+import math
+import os
+from itertools import combinations
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit, softmax
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- rounding
+
+def test_bf16_rounding_golden():
+    for c in _load("bf16_rounding_cases.json")["cases"]:
+        got = float(O.round_to_bf16(np.array([c["value"]]))[0])
+        assert got == c["expect"], c
+
+
+def test_bf16_rounding_matches_library_on_fp32_values():
+    # fp32 -> bf16 is a single rounding in torch (round to nearest even), so on
+    # values exactly representable in fp32 the oracle's one-step rounding must agree.
+    v = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+        rng.integers(-70000, 70000, 5000).astype(np.float64),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.round_to_bf16(v.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bf16_rounding_subnormal_and_overflow():
+    assert O.round_to_bf16(np.array([2.0 ** -133]))[0] == 2.0 ** -133
+    assert O.round_to_bf16(np.array([2.0 ** -135]))[0] == 0.0          # below half spacing
+    assert math.isinf(O.round_to_bf16(np.array([3.5e38]))[0])
+    big = float(torch.tensor(3.38e38).to(torch.bfloat16).item())
+    assert O.round_to_bf16(np.array([big]))[0] == big
+
+
+# ---------------------------------------------------------------- logits
+
+def test_router_logits_match_library_matmul():
+    x = torch.randn(37, 96, dtype=torch.float64).to(torch.bfloat16).to(torch.float64)
+    w = torch.randn(96, 5, dtype=torch.float64).to(torch.bfloat16).to(torch.float64)
+    b = torch.randn(5, dtype=torch.float64).float().double()
+    ref = (x @ w + b).float().numpy()
+    got = O.router_logits(x.numpy(), w.numpy(), b.numpy())
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_router_logits_orientation_and_bias_exact():
+    # Integer inputs: every partial sum is exact, so the result is known exactly.
+    x = np.array([[1, 2, 3]], dtype=np.float64)             # [T=1, H=3]
+    w = np.array([[1, 0], [0, 1], [1, 1]], dtype=np.float64)  # [H=3, E=2]
+    got = O.router_logits(x, w, np.array([0.5, -1.0]))
+    np.testing.assert_array_equal(got, np.array([[4.5, 4.0]], dtype=np.float32))
+
+
+# ---------------------------------------------------------------- top-k
+
+@pytest.mark.parametrize("E", [2, 3, 4, 5, 6, 8])
+def test_topk_matches_bruteforce(E):
+    for k in range(1, min(3, E) + 1):
+        lg = rng.standard_normal((200, E)).astype(np.float32)
+        idx = O.topk_select(lg, k)
+        for t in range(lg.shape[0]):
+            assert tuple(idx[t]) == O.topk_select_bruteforce(lg[t], k)
+            # independent check: the chosen set has the largest sum over all subsets
+            best = max(combinations(range(E), k), key=lambda s: sum(float(lg[t, e]) for e in s))
+            assert set(idx[t]) == set(best)
+
+
+def test_topk_k_equals_E_is_descending_sort():
+    lg = rng.standard_normal((50, 7)).astype(np.float32)
+    idx = O.topk_select(lg, 7)
+    np.testing.assert_array_equal(idx, np.argsort(-lg, axis=1, kind="stable"))
+
+
+def test_topk_k1_is_argmax_with_low_id_ties():
+    lg = rng.integers(0, 3, (300, 6)).astype(np.float32)     # many ties
+    idx = O.topk_select(lg, 1)
+    np.testing.assert_array_equal(idx[:, 0], np.argmax(lg, axis=1))
+
+
+def test_topk_ties_and_nan():
+    lg = np.array([[1.0, 2.0, 2.0, 0.5],
+                   [np.nan, -np.inf, 1.0, np.nan]], dtype=np.float32)
+    idx = O.topk_select(lg, 4)
+    assert list(idx[0]) == [1, 2, 0, 3]
+    assert list(idx[1]) == [2, 1, 0, 3]
+
+
+# ---------------------------------------------------------------- gates
+
+def test_gates_sum_to_one_and_closed_forms():
+    lg = (rng.standard_normal((500, 8)) * 3).astype(np.float32)
+    for k in (1, 2, 3):
+        idx = O.topk_select(lg, k)
+        g = O.topk_gates(lg, idx).astype(np.float64)
+        assert np.all(np.abs(g.sum(1) - 1.0) <= 1e-6)
+        assert np.all(g[:, :-1] >= g[:, 1:])          # descending, like the logits
+        if k == 1:
+            np.testing.assert_array_equal(g[:, 0], 1.0)
+        if k == 2:
+            sel = np.take_along_axis(lg.astype(np.float64), idx.astype(np.int64), 1)
+            np.testing.assert_allclose(g[:, 0], expit(sel[:, 0] - sel[:, 1]), rtol=1e-7)
+
+
+def test_gates_equal_full_softmax_then_renormalise():
+    lg = (rng.standard_normal((300, 16)) * 2).astype(np.float32)
+    idx = O.topk_select(lg, 2)
+    p = softmax(lg.astype(np.float64), axis=1)               # library softmax over all E
+    sel = np.take_along_axis(p, idx.astype(np.int64), 1)
+    ref = sel / sel.sum(1, keepdims=True)
+    np.testing.assert_allclose(O.topk_gates(lg, idx), ref, rtol=1e-7, atol=0)
+    np.testing.assert_allclose(O.topk_gates_literal(lg, idx), ref, rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------- dispatch
+
+def test_capacity_values():
+    assert O.capacity(1.2, 4096, 2, 8) == 1229
+    assert O.capacity(1.25, 32768, 2, 32) == 2560
+    assert O.capacity(0.5, 512, 2, 8) == 64
+    assert O.capacity(1.0, 8, 1, 2) == 4
+    assert O.capacity(0.0, 8, 1, 2) is None
+    assert O.capacity(-1.0, 8, 1, 2) is None
+    # the factor is the float32 the library receives: fp32(1.1) * 10 > 11
+    assert O.capacity(1.1, 10, 1, 1) == 12
+    assert O.capacity(1e-9, 8, 1, 2) == 1
+
+
+@pytest.mark.parametrize("case", _load("capacity_cases.json")["cases"], ids=lambda c: c["name"])
+def test_permute_golden(case):
+    idx = np.array(case["topk_idx"], dtype=np.int32)
+    cap = O.capacity(case["capacity_factor"], case["T"], case["k"], case["E"])
+    assert cap == case["capacity"]
+    p = O.permute(idx, case["E"], cap)
+    for key in ("counts", "kept", "offsets", "row_token", "row_slot", "row_map"):
+        np.testing.assert_array_equal(p[key], np.array(case[key]), err_msg=key)
+    assert p["dropped"] == case["dropped"]
+
+
+def test_counts_match_bincount():
+    idx = rng.integers(0, 13, (1000, 3)).astype(np.int32)
+    np.testing.assert_array_equal(O.expert_counts(idx, 13), np.bincount(idx.ravel(), minlength=13))
+
+
+def test_index_out_of_range_is_an_error():
+    with pytest.raises(O.IndexOutOfRange):
+        O.permute(np.array([[0, 4]], dtype=np.int32), 4, None)
+    with pytest.raises(O.IndexOutOfRange):
+        O.permute(np.array([[-1, 1]], dtype=np.int32), 4, None)
+
+
+def _distinct_ids(T, E, k, skew=0.0):
+    w = np.exp(-skew * np.arange(E)); w /= w.sum()
+    return np.stack([rng.choice(E, size=k, replace=False, p=w) for _ in range(T)]).astype(np.int32)
+
+
+def test_permute_no_limit_is_stable_sort_by_expert():
+    T, E, k = 400, 9, 3
+    idx = _distinct_ids(T, E, k)
+    p = O.permute(idx, E, None)
+    order = np.argsort(idx.ravel(), kind="stable")            # library stable sort
+    np.testing.assert_array_equal(p["row_token"], order // k)
+    np.testing.assert_array_equal(p["row_slot"], order % k)
+    assert p["dropped"] == 0
+
+
+@pytest.mark.parametrize("cf", [0.0, 0.5, 0.8, 1.0, 1.3])
+def test_permute_invariants(cf):
+    T, E, k = 600, 8, 2
+    idx = _distinct_ids(T, E, k, skew=0.3)
+    cap = O.capacity(cf, T, k, E)
+    p = O.permute(idx, E, cap)
+    counts = np.bincount(idx.ravel(), minlength=E)
+    np.testing.assert_array_equal(p["counts"], counts)
+    kept_expected = counts if cap is None else np.minimum(counts, cap)
+    np.testing.assert_array_equal(p["kept"], kept_expected)
+    assert p["R"] == T * k - p["dropped"] == kept_expected.sum()
+    assert np.all(np.diff(p["offsets"]) >= 0) and p["offsets"][0] == 0
+    for e in range(E):
+        seg = p["row_token"][p["offsets"][e]:p["offsets"][e + 1]]
+        assert np.all(np.diff(seg) > 0)                          # stable, one row per token
+        assert np.all(idx[seg, p["row_slot"][p["offsets"][e]:p["offsets"][e + 1]]] == e)
+    # row_map o row_token is the identity on kept rows
+    r = np.arange(p["R"])
+    np.testing.assert_array_equal(p["row_map"][p["row_token"], p["row_slot"]], r)
+    # drops are first-come: a dropped pair's expert already had C earlier pairs kept
+    if cap is not None:
+        for t, s in zip(*np.nonzero(p["row_map"] < 0)):
+            e = idx[t, s]
+            earlier = p["row_token"][p["offsets"][e]:p["offsets"][e + 1]]
+            assert len(earlier) == cap and np.all(earlier < t + (s > 0))
+    # permute then unpermute gives x back on every kept slot
+    x = rng.standard_normal((T, 5))
+    x_perm = x[p["row_token"]]
+    for t in range(T):
+        for s in range(k):
+            if p["row_map"][t, s] >= 0:
+                np.testing.assert_array_equal(x_perm[p["row_map"][t, s]], x[t])
+
+
+# ---------------------------------------------------------------- expert FFN / combine
+
+def test_activations_match_library():
+    z = np.linspace(-8, 8, 1001)
+    zt = torch.from_numpy(z)
+    np.testing.assert_allclose(O.gelu(z), torch.nn.functional.gelu(zt).numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(O.silu(z), torch.nn.functional.silu(zt).numpy(), rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_single_expert_k1_equals_dense_ffn(act):
+    # E=1, k=1, no capacity: every gate is 1 and the layer is the dense FFN.
+    T, H, F = 33, 24, 40                                       # H != F: a transpose fails
+    x = rng.standard_normal((T, H)).astype(np.float32).astype(np.float64)
+    wg = rng.standard_normal((H, 1))
+    w1 = rng.standard_normal((1, H, F)) / math.sqrt(H)
+    w3 = rng.standard_normal((1, H, F)) / math.sqrt(H) if act == "swiglu" else None
+    w2 = rng.standard_normal((1, F, H)) / math.sqrt(F)
+    res = O.moe_forward(x, wg, None, w1, w3, w2, 1, 0.0, act, "f32")
+    xt = torch.from_numpy(x)
+    z1 = xt @ torch.from_numpy(w1[0])
+    if act == "gelu":
+        h = torch.nn.functional.gelu(z1)
+    else:
+        h = torch.nn.functional.silu(z1) * (xt @ torch.from_numpy(w3[0]))
+    ref = (h.float().double() @ torch.from_numpy(w2[0])).numpy()
+    np.testing.assert_array_equal(res["topk_gate"], 1.0)
+    np.testing.assert_allclose(res["out"], ref, rtol=2e-6, atol=2e-6 * np.abs(ref).max())
+
+
+def test_identity_experts_give_x_times_kept_gate_sum():
+    T, H, E, k = 120, 16, 6, 2
+    x = O.round_to_bf16(rng.standard_normal((T, H)))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    for cf in (0.0, 0.6):
+        res = O.moe_forward(x, None, None, None, None, None, k, cf, "identity", "f32", logits=lg)
+        g = res["topk_gate"].astype(np.float64) * (res["row_map"] >= 0)
+        ref = x * g.sum(1, keepdims=True)
+        np.testing.assert_allclose(res["out"], ref, rtol=1e-7, atol=1e-7)
+        if cf == 0.0:
+            np.testing.assert_allclose(res["out"], x, rtol=1e-6, atol=1e-6)
+        else:
+            assert res["dropped"] > 0
+            all_dropped = np.all(res["row_map"] < 0, axis=1)
+            assert np.all(res["out"][all_dropped] == 0)
+
+
+def test_combine_is_linear_in_y():
+    T, H, k = 50, 8, 2
+    row_map = np.arange(T * k).reshape(T, k)
+    row_map[3, 1] = -1
+    g = rng.random((T, k)).astype(np.float32)
+    y1, y2 = rng.standard_normal((T * k, H)), rng.standard_normal((T * k, H))
+    a, b = 0.75, -2.5
+    lhs = O.combine(a * y1 + b * y2, g, row_map, "f32")
+    rhs = a * O.combine(y1, g, row_map, "f32") + b * O.combine(y2, g, row_map, "f32")
+    np.testing.assert_allclose(lhs, rhs, rtol=1e-5, atol=1e-5)
+
+
+def test_layer_matches_per_token_pseudocode():
+    """The grouped (permute -> expert loop -> combine) oracle equals the pages'
+    per-token form: softmax over all experts, top-k, renormalise, sum of
+    gate-weighted expert outputs — written here with torch float64 ops."""
+    T, H, F, E, k = 40, 16, 24, 5, 2
+    x = rng.standard_normal((T, H))
+    wg = rng.standard_normal((H, E))
+    w1 = rng.standard_normal((E, H, F)) / 4
+    w3 = rng.standard_normal((E, H, F)) / 4
+    w2 = rng.standard_normal((E, F, H)) / 5
+    res = O.moe_forward(x, wg, None, w1, w3, w2, k, 0.0, "swiglu", "f32")
+    xt, wgt = torch.from_numpy(x), torch.from_numpy(wg)
+    for t in range(T):
+        logits = (xt[t] @ wgt).float().double()
+        p = torch.softmax(logits, 0)
+        top = torch.topk(p, k)
+        gates = top.values / top.values.sum()
+        acc = torch.zeros(H, dtype=torch.float64)
+        for gi, e in zip(gates, top.indices.tolist()):
+            h = torch.nn.functional.silu(xt[t] @ torch.from_numpy(w1[e])) * (xt[t] @ torch.from_numpy(w3[e]))
+            acc += gi * (h.float().double() @ torch.from_numpy(w2[e])).float().double()
+        assert list(res["topk_idx"][t]) == top.indices.tolist()
+        np.testing.assert_allclose(res["out"][t], acc.numpy(), rtol=1e-5, atol=1e-6)
+
+
+def test_sampled_rows_equal_full_layer():
+    T, H, F, E, k = 64, 16, 32, 4, 2
+    x = O.round_to_bf16(rng.standard_normal((T, H)))
+    wg = O.round_to_bf16(rng.standard_normal((H, E)) / 4)
+    w1 = O.round_to_bf16(rng.standard_normal((E, H, F)) / 4)
+    w2 = O.round_to_bf16(rng.standard_normal((E, F, H)) / 5)
+    for cf in (0.0, 0.7):
+        full = O.moe_forward(x, wg, None, w1, None, w2, k, cf, "gelu", "bf16")
+        toks = np.array([0, 5, 17, 63])
+        samp = O.moe_forward_sampled(x, full["logits"], w1, None, w2, k, cf, "gelu", "bf16", toks)
+        np.testing.assert_array_equal(samp["out_rows"], full["out"][toks])
