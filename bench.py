@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE-layer forward pass on B200 (one JSON line on rank 0).
+
+Metric: MoE-layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; route+permute % HBM.
+
+One step = one whole forward of the layer (route -> permute -> grouped expert
+FFN -> combine) over one batch of seeded synthetic tokens already resident in
+HBM.  The default workload is the page-1 shape (T=4096 = batch 8 x seq 512,
+hidden 2048, 8 GELU experts of ffn 8192, top-2, capacity factor 1.2).
+
+  python bench.py [--gpus N --steps K --warmup W] [--config NAME|1..5] [--impl reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own replica on its
+own tokens (token data-parallel: the layer needs no collective); the reported
+value is the tokens of all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from routing_grouped_expert_moe_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200; grouped-GEMM % bf16 peak; route+permute % HBM"
+DEFAULT_CONFIG = "page1_gelu"
+L2_FLUSH_BYTES = 256 << 20
+SPEC_HBM_GBS = 8000.0       # ~8 TB/s (spec wording of the targets)
+SPEC_BF16_TFLOPS = 2250.0   # dense bf16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of the grouped GEMM kernels from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source they were taken on; None until captured.
+NCU_TRAFFIC = {"source_sha": None, "bytes_per_forward": None}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU seconds for the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+def resolve_config(name: str) -> synth.MoEConfig:
+    if name.isdigit():
+        name = synth.NUMBERED[int(name) - 1]
+    return synth.CONFIGS[name]
+
+
+def workload_desc(cfg: synth.MoEConfig) -> dict:
+    return {"workload": cfg.name, "description": cfg.description, "T": cfg.T, "H": cfg.H,
+            "F": cfg.F, "E": cfg.E, "top_k": cfg.top_k, "act": cfg.act,
+            "capacity_factor": cfg.capacity_factor, "storage": cfg.dtype, "seed": cfg.seed}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm_tcgen05.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "routing_grouped_expert_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- work model
+
+def algorithmic_work(cfg: synth.MoEConfig, counts) -> dict:
+    """Algorithmic FLOPs / bytes of one forward, from the pre-drop expert counts."""
+    s = cfg.elem_bytes
+    T, H, F, E, k = cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k
+    if cfg.capacity_factor > 0:
+        import math
+        cap = math.ceil(float(torch.tensor(cfg.capacity_factor, dtype=torch.float32)) * T * k / E)
+        kept = [min(c, cap) for c in counts]
+    else:
+        kept = list(counts)
+    R = sum(kept)
+    active = sum(1 for c in kept if c > 0)
+    mats = 3 if cfg.act == "swiglu" else 2
+    gemm_flops = 2.0 * R * H * F * mats
+    weight_bytes = active * H * F * mats * s
+    gemm1_flops = 2.0 * R * H * F * (mats - 1)
+    gemm2_flops = 2.0 * R * H * F
+    # GEMM bytes: weights once + A rows in + h out (GEMM-1) + h in + y out (GEMM-2)
+    gemm1_bytes = active * H * F * (mats - 1) * s + R * H * s + R * F * s
+    gemm2_bytes = active * H * F * s + R * F * s + R * H * s
+    route_bytes = T * H * s + H * E * s + T * k * 8 + (E * 4 if cfg.bias != "none" else 0)
+    scan_bytes = 2 * (E + 1) * 4
+    scatter_bytes = T * k * 4 + R * 4 + T * k * 4 + (2 * R * H * s)   # ids, row_token, row_map, x_perm
+    combine_bytes = R * H * s + T * k * 8 + T * H * s
+    return {"R": R, "active_experts": active, "gemm_flops": gemm_flops, "gemm1_flops": gemm1_flops,
+            "gemm2_flops": gemm2_flops, "weight_bytes": weight_bytes, "gemm1_bytes": gemm1_bytes,
+            "gemm2_bytes": gemm2_bytes, "route_bytes": route_bytes, "scan_bytes": scan_bytes,
+            "scatter_bytes": scatter_bytes, "combine_bytes": combine_bytes}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # pragma: no cover
+            self.error = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def stop(self, t0=None, t1=None):
+        self._stop.set()
+        if self._ok:
+            self._t.join(timeout=2)
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "source": "unavailable"}
+        sel = [s for s in self.samples if (t0 is None or s[0] >= t0) and (t1 is None or s[0] <= t1)]
+        if not sel:
+            sel = self.samples
+        mhz = [s[1] for s in sel]
+        bits = 0
+        for s in sel:
+            bits |= int(s[2])
+        reasons = [v for k, v in self.REASONS.items() if bits & k and v != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel), "source": "nvml"}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(cfg: synth.MoEConfig, d: dict, n_tokens: int) -> float:
+    """Seconds the CPU oracle takes for the whole layer on the first n_tokens tokens."""
+    from oracle import moe_oracle as O
+    f = lambda t: None if t is None else t.float().numpy()  # noqa: E731
+    x = f(d["x"][:n_tokens])
+    t0 = time.perf_counter()
+    O.moe_forward(x, d["_wg"], d["_b"], d["_w1"], d["_w3"], d["_w2"], cfg.top_k,
+                  cfg.capacity_factor, cfg.act, cfg.dtype)
+    return time.perf_counter() - t0
+
+
+def _oracle_inputs(cfg, d):
+    f = lambda t: None if t is None else t.float().numpy()  # noqa: E731
+    d["_wg"], d["_b"] = f(d["w_gate"]), f(d["gate_bias"])
+    d["_w1"], d["_w3"], d["_w2"] = f(d["w1"]), f(d["w3"]), f(d["w2"])
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def calibrate_tokens(cfg, d, target_s: float) -> tuple[int, float]:
+    n = min(cfg.T, 64)
+    dt = oracle_sample(cfg, d, n)
+    while dt < 0.25 * target_s and n < cfg.T:
+        n = min(cfg.T, max(n * 2, int(n * target_s / max(dt, 1e-3) * 0.5)))
+        dt = oracle_sample(cfg, d, n)
+    return n, dt
+
+
+def cpu_baseline(cfg, d, target_s: float) -> dict:
+    _oracle_inputs(cfg, d)
+    n, dt = calibrate_tokens(cfg, d, target_s)
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"whole layer (float64 numpy oracle) on the first {n} of {cfg.T} tokens "
+                      f"of {cfg.name}, {dt:.1f} s"}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    d = synth.make_inputs(cfg)
+    _oracle_inputs(cfg, d)
+    # each step: the oracle on a bounded sample sized so K+W steps take ~2 minutes
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    n, _ = calibrate_tokens(cfg, d, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, d, n)
+    times = [oracle_sample(cfg, d, n) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**workload_desc(cfg), "sample_tokens_per_step": n},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{n} of {cfg.T} tokens per step, whole layer"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def main(argv=None):
+    args = parse_args(argv)
+    cfg = resolve_config(args.config)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from routing_grouped_expert_moe_b200 import binding as B
+
+    # inputs: weights shared across ranks (same seed), tokens differ per rank
+    d = synth.make_inputs(cfg)
+    if rank > 0:
+        d["x"] = synth.normal(cfg.seed + 7919 * rank, synth.STREAM_X, (cfg.T, cfg.H), cfg.x_std,
+                              cfg.torch_dtype)
+    g = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    T, H, F, E, k = cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k
+    ws = B.alloc_workspace(B.workspace_bytes(T, H, F, E, k, cfg.act, cfg.torch_dtype), dev)
+    out = torch.empty(T, H, dtype=cfg.torch_dtype, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def fwd(out_counts=None):
+        B.forward(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], k,
+                  cfg.capacity_factor, cfg.act, out=out, ws=ws, expert_counts_out=out_counts)
+
+    # warm-up
+    fwd(counts)
+    torch.cuda.synchronize()
+    st = B.device_status(ws)
+    if st != B.OK:
+        raise RuntimeError(f"device status {B.status_string(st)}")
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize()
+    work = algorithmic_work(cfg, counts.cpu().tolist())
+
+    # ---- headline: K fused forwards, L2 flushed before each, CUDA events per step
+    sampler = ClockSampler(dev.index).start()
+    time.sleep(0.05)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        fwd()
+        ends[i].record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+    ms_per_step = total_ms / args.steps
+    value = T * world * args.steps / (total_ms / 1000.0)
+    gpu_launches = 7 * args.steps
+
+    # ---- per-stage times of the same fused path (events at stage boundaries)
+    n_stage = min(args.steps, 50)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n_stage)]
+    for i in range(n_stage):
+        flush.zero_()
+        B.forward_timed(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], k,
+                        cfg.capacity_factor, cfg.act, out, ws, ev[i])
+    torch.cuda.synchronize()
+    names = ["route", "scan", "scatter", "gemm1", "gemm2", "combine"]
+    stage_ms = {n: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_stage))
+                for j, n in enumerate(names)}
+
+    # ---- end to end through the host-buffer entry point (H2D + layer + D2H)
+    n_e2e = min(args.steps, 50)
+    x_host = d["x"].pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    ws_h = B.alloc_workspace(B.forward_host_workspace_bytes(T, H, F, E, k, cfg.act,
+                                                            cfg.torch_dtype), dev)
+    e2e_ms = []
+    for i in range(n_e2e + 2):
+        flush.zero_()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record()
+        B.forward_host(x_host, g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], k,
+                       cfg.capacity_factor, cfg.act, out_host=out_host, ws=ws_h)
+        s1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            e2e_ms.append(s0.elapsed_time(s1))
+    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = T * world / (float(e2e_t.item()) / 1000.0)
+    io_bytes = T * H * cfg.elem_bytes
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tc_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    gemm_ms = stage_ms["gemm1"] + stage_ms["gemm2"]
+    gemm_tflops = work["gemm_flops"] / (gemm_ms / 1e3) / 1e12
+    rp_bytes = work["route_bytes"] + work["scan_bytes"] + work["scatter_bytes"]
+    rp_ms = stage_ms["route"] + stage_ms["scan"] + stage_ms["scatter"]
+    rp_gbs = rp_bytes / (rp_ms / 1e3) / 1e9
+    comb_gbs = work["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
+    traffic = None
+    if NCU_TRAFFIC["source_sha"] == gemm_source_sha():
+        traffic = NCU_TRAFFIC["bytes_per_forward"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic (seeded Philox normal inputs, random-init weights)",
+        "config": {**workload_desc(cfg),
+                   "l2": "flushed before every step (256 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world} (token data-parallel, no collective)"},
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes, "ms_per_step": float(e2e_t.item()),
+                "entry_point": "moe_forward_host"},
+        "gpu_launches": gpu_launches,
+        "roofline": {"kernel": "k_gemm_tc (expert GEMM-1 + GEMM-2)", "bound": "tensor",
+                     "achieved": gemm_tflops, "peak": tc, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / tc, "peak_source": f"{peak_src} burst bf16",
+                     "frac_of_sustained": gemm_tflops / tc_sus,
+                     "frac_of_spec": gemm_tflops / SPEC_BF16_TFLOPS,
+                     "algorithmic_flops": work["gemm_flops"], "traffic": traffic},
+        "grouped_gemm": {"tflops": gemm_tflops, "frac_measured_peak": gemm_tflops / tc,
+                         "frac_spec_peak": gemm_tflops / SPEC_BF16_TFLOPS,
+                         "gemm1_tflops": work["gemm1_flops"] / (stage_ms["gemm1"] / 1e3) / 1e12,
+                         "gemm2_tflops": work["gemm2_flops"] / (stage_ms["gemm2"] / 1e3) / 1e12},
+        "route_permute": {"gbs": rp_gbs, "frac_measured_hbm": rp_gbs / hbm,
+                          "frac_spec_hbm": rp_gbs / SPEC_HBM_GBS, "bytes": rp_bytes,
+                          "route_gbs": work["route_bytes"] / (stage_ms["route"] / 1e3) / 1e9},
+        "combine": {"gbs": comb_gbs, "frac_measured_hbm": comb_gbs / hbm},
+        "stage_us": {n: 1000.0 * v for n, v in stage_ms.items()},
+        "kept_rows": work["R"],
+        "page_figures_context": {
+            "MoE-32E seq=1024 FP16, Ascend 910": "standard 1850 ms, ops-transformer 620 ms",
+            "routing stage, Ascend 910B": "original 8.2 ms, page's method 1.7 ms"},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, d, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

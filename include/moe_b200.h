@@ -1,0 +1,180 @@
+/*
+ * moe_b200.h — C ABI of the B200 (sm_100a) forward pass of one Mixture-of-Experts layer.
+ *
+ * The layer (router -> permute -> grouped expert FFN -> combine) is the one the
+ * following pages describe; each entry point cites the passage that defines it:
+ *   [P2] "MoE模型高效推理：CANN算子库优化实践" (intelliparadigm.com)
+ *   [P3] "ops-transformer 仓库 - MoE 算子优化实战" (gitcode.csdn.net)
+ *   [P4] lshu.cn/news/82007: calling the MoE fused operators through torch_npu
+ *   [P1] hnwysp.cn/news/132341: ops-transformer MoE operator optimisation
+ *   [P5] "ops-transformer 算子精讲：昇腾 NPU 上的注意力机制与融合算子实现" (mhpn.cn)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Ownership: the caller allocates and frees every buffer.  The library never
+ *   allocates device memory; scratch comes from a caller-provided workspace
+ *   `ws` of at least moe_workspace_bytes(...) bytes (256-byte aligned).
+ * Pointers: device pointers unless stated otherwise, 16-byte aligned.
+ * Layouts: dense row-major.  x[T,H]; w_gate[H,E]; w1,w3[E,H,F]; w2[E,F,H];
+ *   topk_idx / topk_gate / row_map [T,top_k]; x_perm, y [rows,H]; h [rows,F].
+ *   T tokens, H hidden, F expert intermediate size, E experts.
+ * Element type: MOE_BF16 (bf16 storage, fp32 accumulation, tensor cores) or
+ *   MOE_F32 (fp32 storage and arithmetic on CUDA cores, no TF32).
+ * Asynchrony: every call is enqueued on `stream` and returns at once.
+ *   Argument errors are detected on the host and returned before any launch.
+ *   Errors found by kernels (an expert id outside [0,E), a pipeline wait that
+ *   timed out) are written to a status word at the start of `ws`; read it with
+ *   moe_get_device_status().
+ * Limits: 1 <= top_k <= 8, top_k <= E <= 256, H and F multiples of 8,
+ *   T*top_k*max(H,F) < 2^31.  Violations return MOE_ERR_INVALID_ARG or
+ *   MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, bad size or enum          */
+  MOE_ERR_INDEX_OUT_OF_RANGE = 2,  /* an expert id outside [0,E) ([P4] §5.2, §7)          */
+  MOE_ERR_WORKSPACE = 3,           /* ws smaller than moe_workspace_bytes()               */
+  MOE_ERR_UNSUPPORTED = 4,         /* sizes outside the limits above                      */
+  MOE_ERR_CUDA = 5,                /* a CUDA runtime or driver call failed                */
+  MOE_ERR_TIMEOUT = 6              /* a kernel's bounded pipeline wait ran out            */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+  MOE_ACT_SWIGLU = 0,   /* h = silu(x W1) * (x W3)                                        */
+  MOE_ACT_GELU = 1,     /* h = gelu(x W1), exact erf form; w3 unused                      */
+  MOE_ACT_IDENTITY = 2  /* test experts: y = x (weights unused)                           */
+} moe_act;
+
+typedef void* moe_stream_t;  /* a cudaStream_t; NULL = the legacy default stream */
+
+/* Bytes of workspace that every entry point below needs for these sizes
+ * (the fused moe_forward needs the most; one size serves every call).     */
+size_t moe_workspace_bytes(int T, int H, int F, int E, int top_k, moe_act act, moe_dtype dt);
+
+/* Router.  [P2] §2.1 (gates = softmax(x @ W_gate), top_k(gates, k=2)), §3.2.1
+ * (renormalise the kept experts); [P5] ch.8 (normalize_scores=True).
+ *   logits[t,e] = sum_h x[t,h] W_gate[h,e] + gate_bias[e]   (fp32 accumulate)
+ *   topk_idx[t,0..k-1]: the k largest logits, slot 0 the largest; ties go to the
+ *     lower expert id; NaN ranks below -inf.
+ *   topk_gate[t,s] = exp(l_s - l_0) / sum_j exp(l_j - l_0) over the k selected
+ *     (softmax over all E renormalised over the top-k).
+ * gate_bias (fp32 [E]) and logits_out (fp32 [T,E]) may be NULL.           */
+moe_status moe_route(const void* x, const void* w_gate, const float* gate_bias,
+                     int T, int H, int E, int top_k, moe_dtype dt,
+                     int32_t* topk_idx, float* topk_gate, float* logits_out,
+                     moe_stream_t stream);
+
+/* Selection and gates only, from caller-given fp32 logits [T,E]; same rules as
+ * moe_route.  Lets a caller check selection on identical logits.           */
+moe_status moe_route_from_logits(const float* logits, int T, int E, int top_k,
+                                 int32_t* topk_idx, float* topk_gate, moe_stream_t stream);
+
+/* Permute / dispatch.  [P4] §4 (npu_moe_token_preprocess: token rearrangement),
+ * §5.2 (int32 expert ids in [0,E)), §5.3 (fixed per-expert buffer); [P1] §3.2
+ * (capacity_factor); [P3] SparseGather.
+ *   expert_counts[e]  (pre-drop) = #{(t,s): token_expert_idx[t,s] = e}
+ *   C = ceil(capacity_factor * T * top_k / E); no limit when capacity_factor <= 0
+ *   Pairs (t,s) are walked in token order, then slot order; a pair is kept when
+ *   fewer than C pairs of its expert were kept before it.
+ *   expert_offsets[E+1]: exclusive prefix sum of kept counts; R = offsets[E].
+ *   Kept pair (t,s) of expert e goes to row offsets[e] + (its arrival rank):
+ *     row_token[row] = t, row_map[t,s] = row; dropped pairs get row_map = -1.
+ *   x_perm (optional, [T*top_k,H]): x_perm[row] = x[row_token[row]].
+ * Out-of-range ids are not clamped: they count as dropped and the device
+ * status becomes MOE_ERR_INDEX_OUT_OF_RANGE.  x may be NULL when x_perm is.
+ * row_token must hold T*top_k entries (only the first R are written).      */
+moe_status moe_permute(const void* x, const int32_t* token_expert_idx,
+                       int T, int H, int E, int top_k, float capacity_factor, moe_dtype dt,
+                       void* x_perm, int32_t* expert_counts, int32_t* expert_offsets,
+                       int32_t* row_token, int32_t* row_map,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped expert FFN.  [P4] §3 (x times expert_weight[num_experts, hidden,
+ * intermediate], then activation and down-projection), §4 (npu_moe_matmul);
+ * [P1] §2.2 (one batched GEMM instead of one launch per expert).
+ * For every expert e and row r in [offsets[e], offsets[e+1]):
+ *   a_r = x_perm[r]            when row_token == NULL
+ *       = x[row_token[r]]      otherwise (rows gathered on the fly; x_perm unused)
+ *   h_r = act(a_r W1[e] [, a_r W3[e]])  rounded to dt
+ *   y_r = h_r W2[e]                     rounded to dt
+ * T is the row count of x (for the gathered form).  y has R_max >= R rows;
+ * rows >= R are not written.  R is read on the device from expert_offsets[E]
+ * (no host synchronisation).  h lives in ws.                                */
+moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const void* x,
+                           const void* w1, const void* w3, const void* w2,
+                           const int32_t* expert_offsets, int R_max, int T, int H, int F,
+                           int E, moe_act act, moe_dtype dt, void* y,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Deterministic weighted combine.  [P2] §2.1 (sum of gate-weighted expert
+ * outputs); [P3] SparseScatterAdd; [P4] §4 (npu_moe_token_postprocess).
+ *   out[t] = sum_{s=0..k-1, row_map[t,s] >= 0} topk_gate[t,s] * y[row_map[t,s]]
+ * summed in slot order in fp32 and rounded once to dt; no atomics, so the
+ * result is bit-identical from run to run.                                  */
+moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
+                                 int T, int H, int top_k, moe_dtype dt, void* out,
+                                 moe_stream_t stream);
+
+/* The whole layer: route -> permute -> grouped FFN -> combine, enqueued on one
+ * stream with no host synchronisation.  [P3] MoEOperator::Forward; [P5] ch.8
+ * moe_router(x, router_weight, expert_weights, top_k, normalize_scores=True,
+ * capacity_factor); [P4] §1 (fusing permute, matmul, softmax, experts, combine).
+ * topk_idx_out [T,k] and expert_counts_out [E] (pre-drop) may be NULL.      */
+moe_status moe_forward(const void* x, const void* w_gate, const float* gate_bias,
+                       const void* w1, const void* w3, const void* w2,
+                       int T, int H, int F, int E, int top_k, float capacity_factor,
+                       moe_act act, moe_dtype dt, void* out,
+                       int32_t* topk_idx_out, int32_t* expert_counts_out,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward that also records CUDA events at its stage boundaries, for
+ * measuring each kernel of the fused path on the stream it runs on.
+ * events: n_events (>= 7) cudaEvent_t handles; events[i] is recorded before
+ * stage i and events[6] after the last: route (0-1), offsets scan (1-2),
+ * scatter (2-3), expert GEMM-1 (3-4), expert GEMM-2 (4-5), combine (5-6).  */
+moe_status moe_forward_timed(const void* x, const void* w_gate, const float* gate_bias,
+                             const void* w1, const void* w3, const void* w2,
+                             int T, int H, int F, int E, int top_k, float capacity_factor,
+                             moe_act act, moe_dtype dt, void* out,
+                             void* ws, size_t ws_bytes, moe_stream_t stream,
+                             void* const* events, int n_events);
+
+/* moe_forward with x and out in HOST memory (page-locked for asynchronous
+ * copies): copies x into the workspace, runs the layer, copies out back, all on
+ * `stream`.  The caller synchronises the stream before reading out_host.
+ * ws must hold moe_forward_host_workspace_bytes(...) bytes.                 */
+size_t moe_forward_host_workspace_bytes(int T, int H, int F, int E, int top_k, moe_act act,
+                                        moe_dtype dt);
+moe_status moe_forward_host(const void* x_host, const void* w_gate, const float* gate_bias,
+                            const void* w1, const void* w3, const void* w2,
+                            int T, int H, int F, int E, int top_k, float capacity_factor,
+                            moe_act act, moe_dtype dt, void* out_host,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, then returns the status the kernels of the last
+ * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */
+moe_status moe_get_device_status(void* ws, moe_stream_t stream);
+
+/* A constant string naming the status code. */
+const char* moe_status_string(moe_status s);
+
+/* Library build tag (architecture and version). */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

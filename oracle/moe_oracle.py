@@ -363,18 +363,25 @@ def moe_forward_sampled(x, logits, w1, w3, w2, top_k: int, capacity_factor: floa
     cap = capacity(capacity_factor, T, top_k, E)
     perm = permute(idx, E, cap)
     tokens = np.asarray(tokens, dtype=np.int64)
-    out_rows = np.zeros((len(tokens), x.shape[1]), dtype=np.float64)
+    H = x.shape[1]
+    # expert outputs of the sampled tokens' kept slots, one expert at a time
+    yrows = {}
+    for e in range(E):
+        pairs = [(int(t), s) for t in tokens for s in range(top_k)
+                 if perm["row_map"][t, s] >= 0 and int(idx[t, s]) == e]
+        if not pairs:
+            continue
+        xe = np.stack([np.asarray(x[t], dtype=np.float64) for t, _ in pairs])
+        ye = expert_ffn(xe, None if w1 is None else w1[e], None if w3 is None else w3[e],
+                        None if w2 is None else w2[e], act, dtype)
+        for (t, s), yr in zip(pairs, ye):
+            yrows[(t, s)] = yr
+    out_rows = np.zeros((len(tokens), H), dtype=np.float64)
     for i, t in enumerate(tokens):
-        acc = np.zeros(x.shape[1], dtype=np.float64)
+        acc = np.zeros(H, dtype=np.float64)
         for s in range(top_k):
-            r = perm["row_map"][t, s]
-            if r < 0:
-                continue
-            e = int(idx[t, s])
-            yrow = expert_ffn(x[t:t + 1], None if w1 is None else w1[e],
-                              None if w3 is None else w3[e], None if w2 is None else w2[e],
-                              act, dtype)[0]
-            acc += float(gates[t, s]) * yrow
+            if (int(t), s) in yrows:
+                acc += float(gates[t, s]) * yrows[(int(t), s)]
         out_rows[i] = round_to(dtype, acc)
     return {"topk_idx": idx, "topk_gate": gates, "capacity": cap, "out_rows": out_rows,
             "tokens": tokens, **perm}

@@ -7,14 +7,12 @@ hand-written sm_100a kernels behind a C ABI (``include/moe_b200.h``).
 The ops live in :mod:`routing_grouped_expert_moe_b200.binding`; importing them
 loads ``lib/libmoe_b200.so`` and raises if it has not been built.
 """
+import importlib
+
 __all__ = ["binding", "synth"]
 
 
 def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    if name == "synth":
-        from . import synth
-        return synth
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

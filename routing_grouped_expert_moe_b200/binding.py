@@ -1,0 +1,294 @@
+"""Python binding of the C ABI in include/moe_b200.h (ctypes; argument marshalling only).
+
+Every function here checks tensor dtypes, devices, shapes and contiguity, turns
+tensors into raw pointers and calls the entry point of the same name on the
+current CUDA stream.  All arithmetic happens in the CUDA library; there is no
+fallback: importing this module raises if ``lib/libmoe_b200.so`` is missing.
+
+Tensors are allocated with torch (PyTorch is used for device memory and streams
+only).  Expert ids are int32, as the MoE fused operators require (an int64
+index tensor is rejected, lshu.cn torch_npu article §5.2).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m routing_grouped_expert_moe_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes (moe_status)
+OK, ERR_INVALID_ARG, ERR_INDEX_OUT_OF_RANGE, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, \
+    ERR_TIMEOUT = range(7)
+F32, BF16 = 0, 1
+ACT = {"swiglu": 0, "gelu": 1, "identity": 2}
+
+_p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "moe_forward_host_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "moe_route": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
+    "moe_route_from_logits": (_i, [_p, _i, _i, _i, _p, _p, _p]),
+    "moe_permute": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_grouped_ffn": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _sz,
+                             _p]),
+    "moe_unpermute_combine": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
+    "moe_forward": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _p, _p, _p,
+                         _sz, _p]),
+    "moe_forward_timed": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _p,
+                               _sz, _p, _p, _i]),
+    "moe_forward_host": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _p, _sz,
+                              _p]),
+    "moe_get_device_status": (_i, [_p, _p]),
+    "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def status_string(s: int) -> str:
+    return _lib.moe_status_string(int(s)).decode()
+
+
+def version() -> str:
+    return _lib.moe_version().decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise MoEError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported element type {t.dtype} (bf16 or fp32)")
+
+
+def _need(t, name, dtype=None, dim=None, cuda=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def workspace_bytes(T, H, F, E, top_k, act="swiglu", dtype=torch.bfloat16) -> int:
+    return int(_lib.moe_workspace_bytes(T, H, F, E, top_k, ACT[act],
+                                        BF16 if dtype == torch.bfloat16 else F32))
+
+
+def forward_host_workspace_bytes(T, H, F, E, top_k, act="swiglu", dtype=torch.bfloat16) -> int:
+    return int(_lib.moe_forward_host_workspace_bytes(T, H, F, E, top_k, ACT[act],
+                                                     BF16 if dtype == torch.bfloat16 else F32))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def route(x, w_gate, gate_bias=None, top_k=2, logits_out=False):
+    """Router: returns (topk_idx int32 [T,k], topk_gate fp32 [T,k][, logits fp32 [T,E]])."""
+    _need(x, "x", dim=2)
+    _need(w_gate, "w_gate", dtype=x.dtype, dim=2)
+    T, H = x.shape
+    E = w_gate.shape[1]
+    if gate_bias is not None:
+        _need(gate_bias, "gate_bias", dtype=torch.float32, dim=1)
+    idx = torch.empty(T, top_k, dtype=torch.int32, device=x.device)
+    gate = torch.empty(T, top_k, dtype=torch.float32, device=x.device)
+    lg = torch.empty(T, E, dtype=torch.float32, device=x.device) if logits_out else None
+    _check(_lib.moe_route(_ptr(x), _ptr(w_gate), _ptr(gate_bias), T, H, E, top_k, _dt(x),
+                          _ptr(idx), _ptr(gate), _ptr(lg), _stream()), "moe_route")
+    return (idx, gate, lg) if logits_out else (idx, gate)
+
+
+def route_from_logits(logits, top_k):
+    _need(logits, "logits", dtype=torch.float32, dim=2)
+    T, E = logits.shape
+    idx = torch.empty(T, top_k, dtype=torch.int32, device=logits.device)
+    gate = torch.empty(T, top_k, dtype=torch.float32, device=logits.device)
+    _check(_lib.moe_route_from_logits(_ptr(logits), T, E, top_k, _ptr(idx), _ptr(gate),
+                                      _stream()), "moe_route_from_logits")
+    return idx, gate
+
+
+def permute(token_expert_idx, num_experts, capacity_factor=0.0, x=None, ws=None):
+    """Dispatch: returns dict(counts, offsets, row_token, row_map[, x_perm])."""
+    _need(token_expert_idx, "token_expert_idx", dtype=torch.int32, dim=2)
+    T, k = token_expert_idx.shape
+    dev = token_expert_idx.device
+    E = int(num_experts)
+    if x is not None:
+        _need(x, "x", dim=2)
+        H, dt = x.shape[1], _dt(x)
+    else:
+        H, dt = 8, BF16
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_token = torch.full((T * k,), -1, dtype=torch.int32, device=dev)
+    row_map = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, H, dtype=x.dtype, device=dev) if x is not None else None
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(T, H, 8, E, k, "identity",
+                                             torch.bfloat16 if dt == BF16 else torch.float32), dev)
+    _check(_lib.moe_permute(_ptr(x), _ptr(token_expert_idx), T, H, E, k,
+                            ctypes.c_float(capacity_factor), dt, _ptr(x_perm), _ptr(counts),
+                            _ptr(offsets), _ptr(row_token), _ptr(row_map), _ptr(ws), ws.numel(),
+                            _stream()), "moe_permute")
+    out = {"counts": counts, "offsets": offsets, "row_token": row_token, "row_map": row_map,
+           "ws": ws}
+    if x_perm is not None:
+        out["x_perm"] = x_perm
+    return out
+
+
+def grouped_ffn(expert_offsets, w1, w3, w2, act="swiglu", x_perm=None, x=None, row_token=None,
+                R_max=None, ws=None, y=None):
+    """Grouped expert FFN over expert-ordered rows; returns y [R_max, H]."""
+    _need(expert_offsets, "expert_offsets", dtype=torch.int32, dim=1)
+    E = expert_offsets.numel() - 1
+    if row_token is not None:
+        _need(row_token, "row_token", dtype=torch.int32)
+        src = _need(x, "x", dim=2)
+        R_max = int(R_max if R_max is not None else row_token.numel())
+    else:
+        src = _need(x_perm, "x_perm", dim=2)
+        R_max = int(R_max if R_max is not None else x_perm.shape[0])
+    H = src.shape[1]
+    T = x.shape[0] if x is not None else 0
+    if act == "identity":
+        F = 8
+    else:
+        _need(w1, "w1", dtype=src.dtype, dim=3)
+        _need(w2, "w2", dtype=src.dtype, dim=3)
+        if act == "swiglu":
+            _need(w3, "w3", dtype=src.dtype, dim=3)
+        F = w1.shape[2]
+    if y is None:
+        y = torch.empty(R_max, H, dtype=src.dtype, device=src.device)
+    if ws is None:
+        ws = alloc_workspace(256 + R_max * F * src.element_size(), src.device)
+    _check(_lib.moe_grouped_ffn(_ptr(x_perm), _ptr(row_token), _ptr(x), _ptr(w1), _ptr(w3),
+                                _ptr(w2), _ptr(expert_offsets), R_max, T, H, F, E, ACT[act],
+                                _dt(src), _ptr(y), _ptr(ws), ws.numel(), _stream()),
+           "moe_grouped_ffn")
+    return y
+
+
+def unpermute_combine(y, topk_gate, row_map, out=None):
+    _need(y, "y", dim=2)
+    _need(topk_gate, "topk_gate", dtype=torch.float32, dim=2)
+    _need(row_map, "row_map", dtype=torch.int32, dim=2)
+    T, k = row_map.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=y.dtype, device=y.device)
+    _check(_lib.moe_unpermute_combine(_ptr(y), _ptr(topk_gate), _ptr(row_map), T, H, k, _dt(y),
+                                      _ptr(out), _stream()), "moe_unpermute_combine")
+    return out
+
+
+def forward(x, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0.0, act="swiglu",
+            out=None, ws=None, topk_idx_out=None, expert_counts_out=None):
+    """The whole layer; returns out [T,H] (same dtype as x)."""
+    _need(x, "x", dim=2)
+    _need(w_gate, "w_gate", dtype=x.dtype, dim=2)
+    T, H = x.shape
+    E = w_gate.shape[1]
+    if gate_bias is not None:
+        _need(gate_bias, "gate_bias", dtype=torch.float32, dim=1)
+    if act == "identity":
+        F = 8
+    else:
+        _need(w1, "w1", dtype=x.dtype, dim=3)
+        _need(w2, "w2", dtype=x.dtype, dim=3)
+        if act == "swiglu":
+            _need(w3, "w3", dtype=x.dtype, dim=3)
+        F = w1.shape[2]
+    if out is None:
+        out = torch.empty_like(x)
+    if ws is None:
+        ws = alloc_workspace(workspace_bytes(T, H, F, E, top_k, act, x.dtype), x.device)
+    if topk_idx_out is not None:
+        _need(topk_idx_out, "topk_idx_out", dtype=torch.int32)
+    if expert_counts_out is not None:
+        _need(expert_counts_out, "expert_counts_out", dtype=torch.int32)
+    _check(_lib.moe_forward(_ptr(x), _ptr(w_gate), _ptr(gate_bias), _ptr(w1), _ptr(w3), _ptr(w2),
+                            T, H, F, E, top_k, ctypes.c_float(capacity_factor), ACT[act], _dt(x),
+                            _ptr(out), _ptr(topk_idx_out), _ptr(expert_counts_out), _ptr(ws),
+                            ws.numel(), _stream()), "moe_forward")
+    return out
+
+
+def forward_timed(x, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor, act, out, ws,
+                  events):
+    """moe_forward recording 7 torch.cuda.Event objects at its stage boundaries."""
+    handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    T, H = x.shape
+    E = w_gate.shape[1]
+    F = 8 if act == "identity" else w1.shape[2]
+    _check(_lib.moe_forward_timed(_ptr(x), _ptr(w_gate), _ptr(gate_bias), _ptr(w1), _ptr(w3),
+                                  _ptr(w2), T, H, F, E, top_k, ctypes.c_float(capacity_factor),
+                                  ACT[act], _dt(x), _ptr(out), _ptr(ws), ws.numel(), _stream(),
+                                  handles, len(events)), "moe_forward_timed")
+    return out
+
+
+def forward_host(x_host, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0.0,
+                 act="swiglu", out_host=None, ws=None):
+    """The whole layer with x and out in page-locked host memory (copies on the stream)."""
+    _need(x_host, "x_host", dim=2, cuda=False)
+    T, H = x_host.shape
+    E = w_gate.shape[1]
+    F = 8 if act == "identity" else w1.shape[2]
+    if out_host is None:
+        out_host = torch.empty_like(x_host, pin_memory=True)
+    if ws is None:
+        ws = alloc_workspace(forward_host_workspace_bytes(T, H, F, E, top_k, act, x_host.dtype),
+                             w_gate.device)
+    _check(_lib.moe_forward_host(_ptr(x_host), _ptr(w_gate), _ptr(gate_bias), _ptr(w1), _ptr(w3),
+                                 _ptr(w2), T, H, F, E, top_k, ctypes.c_float(capacity_factor),
+                                 ACT[act], _dt(x_host), _ptr(out_host), _ptr(ws), ws.numel(),
+                                 _stream()), "moe_forward_host")
+    return out_host
+
+
+def device_status(ws) -> int:
+    """Synchronises the current stream and returns (and clears) the kernels' status word."""
+    return int(_lib.moe_get_device_status(_ptr(ws), _stream()))

@@ -1,0 +1,437 @@
+// C ABI of the MoE layer (declared in include/moe_b200.h): argument checks,
+// workspace layout and the launch sequence of each entry point.  No entry
+// point allocates device memory or synchronises the stream (except
+// moe_get_device_status, whose job is to synchronise).
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.h"
+#include "moe_b200.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+int elem_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+int num_sms_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace: [status | topk_idx | topk_gate | tile_counts | counts | offsets |
+//             row_token | row_map | x_perm | h | y | x_stage | out_stage]
+struct WsLayout {
+  size_t status, topk_idx, topk_gate, tile_counts, counts, offsets, row_token, row_map, x_perm,
+      h, y, x_stage, out_stage, total;
+};
+
+WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt, bool host_stage) {
+  WsLayout L{};
+  const size_t eb = elem_bytes(dt);
+  const size_t R = static_cast<size_t>(T) * k;
+  const size_t tiles = static_cast<size_t>(T) / 16 + 1;  // finest token tiling used
+  size_t o = 0;
+  L.status = o;      o = align_up(o + 4);
+  L.topk_idx = o;    o = align_up(o + R * 4);
+  L.topk_gate = o;   o = align_up(o + R * 4);
+  L.tile_counts = o; o = align_up(o + tiles * E * 4);
+  L.counts = o;      o = align_up(o + static_cast<size_t>(E) * 4);
+  L.offsets = o;     o = align_up(o + static_cast<size_t>(E + 1) * 4);
+  L.row_token = o;   o = align_up(o + R * 4);
+  L.row_map = o;     o = align_up(o + R * 4);
+  L.x_perm = o;      o = align_up(o + R * H * eb);
+  L.h = o;           o = align_up(o + (act == MOE_ACT_IDENTITY ? 0 : R * F * eb));
+  L.y = o;           o = align_up(o + R * H * eb);
+  if (host_stage) {
+    L.x_stage = o;   o = align_up(o + static_cast<size_t>(T) * H * eb);
+    L.out_stage = o; o = align_up(o + static_cast<size_t>(T) * H * eb);
+  }
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status check_common(int T, int H, int E, int k, moe_dtype dt) {
+  if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+bool index_range_ok(int T, int k, int width) {
+  return static_cast<long long>(T) * k * width < (1LL << 31);
+}
+
+int capacity_of(float cf, int T, int k, int E) {
+  if (!(cf > 0.f)) return INT32_MAX;
+  const double c = std::ceil(static_cast<double>(cf) * static_cast<double>(T) * k / E);
+  if (c >= static_cast<double>(INT32_MAX)) return INT32_MAX;
+  return c < 1.0 ? 1 : static_cast<int>(c);
+}
+
+cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Grouped FFN on prepared buffers (shared by moe_grouped_ffn and moe_forward).
+moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, const void* w1,
+                   const void* w3, const void* w2, const int32_t* offsets, int R_max, int T,
+                   int H, int F, int E, moe_act act, moe_dtype dt, void* y, void* h, int* status,
+                   cudaStream_t s, cudaEvent_t mid_event = nullptr) {
+  const int nsm = num_sms_current();
+  const bool gather = row_token != nullptr;
+  const void* a_src = gather ? x : x_perm;
+  const int a_rows = gather ? T : R_max;
+  GemmArgs g{};
+  g.offsets = offsets;
+  g.E = E;
+  g.R_max = R_max;
+  g.T = T;
+  g.status = status;
+  if (act == MOE_ACT_IDENTITY) {
+    g.row_token = row_token;
+    g.N = H;
+    g.K = H;
+    g.out = y;
+    if (launch_copy_rows(a_src, g, elem_bytes(dt), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(mid_event ? cudaEventRecord(mid_event, s) : cudaSuccess);
+  }
+  const int mode1 = act == MOE_ACT_SWIGLU ? 1 : 0;
+  // GEMM-1: h = act(A W1 [, A W3])
+  g.row_token = row_token;
+  g.N = F;
+  g.K = H;
+  g.out = h;
+  cudaError_t err;
+  if (dt == MOE_BF16)
+    err = launch_gemm_tc(mode1, gather, a_src, a_rows, w1, w3, g, nsm, s);
+  else
+    err = launch_gemm_simt(mode1, a_src, w1, w3, g, nsm, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // GEMM-2: y = h W2 (rows already in expert order)
+  g.row_token = nullptr;
+  g.N = H;
+  g.K = F;
+  g.out = y;
+  if (dt == MOE_BF16)
+    err = launch_gemm_tc(2, false, h, R_max, w2, nullptr, g, nsm, s);
+  else
+    err = launch_gemm_simt(2, h, w2, nullptr, g, nsm, s);
+  return cuda_status(err);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(int T, int H, int F, int E, int top_k, moe_act act, moe_dtype dt) {
+  if (T < 0 || H <= 0 || F <= 0 || E <= 0 || top_k <= 0) return 0;
+  return ws_layout(T, H, F, E, top_k, act, dt, false).total;
+}
+
+size_t moe_forward_host_workspace_bytes(int T, int H, int F, int E, int top_k, moe_act act,
+                                        moe_dtype dt) {
+  if (T < 0 || H <= 0 || F <= 0 || E <= 0 || top_k <= 0) return 0;
+  return ws_layout(T, H, F, E, top_k, act, dt, true).total;
+}
+
+moe_status moe_route(const void* x, const void* w_gate, const float* gate_bias, int T, int H,
+                     int E, int top_k, moe_dtype dt, int32_t* topk_idx, float* topk_gate,
+                     float* logits_out, moe_stream_t stream) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_gate || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, 1, H) || !index_range_ok(T, 1, E)) return MOE_ERR_UNSUPPORTED;
+  RouteArgs a{};
+  a.x = x; a.wg = w_gate; a.bias = gate_bias;
+  a.T = T; a.H = H; a.E = E; a.top_k = top_k; a.dt_bf16 = dt == MOE_BF16;
+  a.topk_idx = topk_idx; a.topk_gate = topk_gate; a.logits_out = logits_out;
+  a.tile_counts = nullptr;
+  const RoutePlan p = route_plan(T, H, E, a.dt_bf16, num_sms_current());
+  return cuda_status(launch_route(a, p, as_stream(stream)));
+}
+
+moe_status moe_route_from_logits(const float* logits, int T, int E, int top_k, int32_t* topk_idx,
+                                 float* topk_gate, moe_stream_t stream) {
+  if (T < 0 || E <= 0 || top_k <= 0 || top_k > E) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, 1, E)) return MOE_ERR_UNSUPPORTED;
+  RouteArgs a{};
+  a.T = T; a.E = E; a.top_k = top_k;
+  a.topk_idx = topk_idx; a.topk_gate = topk_gate;
+  return cuda_status(launch_route_from_logits(a, logits, as_stream(stream)));
+}
+
+moe_status moe_permute(const void* x, const int32_t* token_expert_idx, int T, int H, int E,
+                       int top_k, float capacity_factor, moe_dtype dt, void* x_perm,
+                       int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
+                       int32_t* row_map, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (!token_expert_idx || !expert_counts || !expert_offsets || !row_token || !row_map || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, top_k, H)) return MOE_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(T, H, 8, E, top_k, MOE_ACT_IDENTITY, dt, false);
+  if (ws_bytes < L.tile_counts + (static_cast<size_t>(T) / 16 + 1) * E * 4)
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  int* status = at<int>(ws, L.status);
+  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  PermuteArgs p{};
+  p.idx = token_expert_idx;
+  p.T = T; p.k = top_k; p.E = E;
+  p.BT = kPermuteBT;
+  p.tiles = (T + kPermuteBT - 1) / kPermuteBT;
+  p.cap = capacity_of(capacity_factor, T, top_k, E);
+  p.tile_counts = at<int>(ws, L.tile_counts);
+  p.counts = expert_counts; p.offsets = expert_offsets;
+  p.row_token = row_token; p.row_map = row_map;
+  p.x = x; p.x_perm = x_perm; p.H = H; p.elem_bytes = elem_bytes(dt);
+  p.status = status;
+  if (T == 0) {
+    // no pairs: counts are zero, every offset is zero
+    if (cudaMemsetAsync(expert_counts, 0, E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(cudaMemsetAsync(expert_offsets, 0, (E + 1) * 4, s));
+  }
+  if (launch_hist(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_scan(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_scatter(p, s));
+}
+
+moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const void* x,
+                           const void* w1, const void* w3, const void* w2,
+                           const int32_t* expert_offsets, int R_max, int T, int H, int F, int E,
+                           moe_act act, moe_dtype dt, void* y, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU && act != MOE_ACT_IDENTITY)
+    return MOE_ERR_INVALID_ARG;
+  if (R_max < 0 || T < 0 || H <= 0 || F <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0 || F % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets || !y || !ws) return MOE_ERR_INVALID_ARG;
+  const bool gather = row_token != nullptr;
+  const void* a_src = gather ? x : x_perm;
+  if (!a_src || !aligned16(a_src) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (act != MOE_ACT_IDENTITY) {
+    if (!w1 || !w2 || !aligned16(w1) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
+    if (act == MOE_ACT_SWIGLU && (!w3 || !aligned16(w3))) return MOE_ERR_INVALID_ARG;
+  }
+  if (gather && T <= 0) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(R_max, 1, H > F ? H : F)) return MOE_ERR_UNSUPPORTED;
+  if (R_max == 0) return MOE_OK;
+  // h needs R_max * F elements after the status word.
+  const size_t h_off = align_up(4);
+  const size_t need = h_off + static_cast<size_t>(R_max) * F * elem_bytes(dt);
+  if (act != MOE_ACT_IDENTITY && ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < h_off) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  int* status = at<int>(ws, 0);
+  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return run_ffn(x_perm, row_token, x, w1, w3, w2, expert_offsets, R_max, T, H, F, E, act, dt, y,
+                 at<void>(ws, h_off), status, s);
+}
+
+moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
+                                 int T, int H, int top_k, moe_dtype dt, void* out,
+                                 moe_stream_t stream) {
+  if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0 || top_k <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!y || !topk_gate || !row_map || !out || !aligned16(y) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, top_k, H)) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(launch_combine(y, topk_gate, row_map, T, H, top_k, dt == MOE_BF16, out,
+                                    num_sms_current(), as_stream(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bias, const void* w1,
+                        const void* w3, const void* w2, int T, int H, int F, int E, int top_k,
+                        float capacity_factor, moe_act act, moe_dtype dt, void* out,
+                        int32_t* topk_idx_out, int32_t* expert_counts_out, void* ws,
+                        size_t ws_bytes, moe_stream_t stream, cudaEvent_t const* ev) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU && act != MOE_ACT_IDENTITY)
+    return MOE_ERR_INVALID_ARG;
+  if (F <= 0 || F % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_gate || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (act != MOE_ACT_IDENTITY) {
+    if (!w1 || !w2 || !aligned16(w1) || !aligned16(w2)) return MOE_ERR_INVALID_ARG;
+    if (act == MOE_ACT_SWIGLU && (!w3 || !aligned16(w3))) return MOE_ERR_INVALID_ARG;
+  }
+  if (!index_range_ok(T, top_k, H > F ? H : F) || !index_range_ok(T, 1, E))
+    return MOE_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false);
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+
+  cudaStream_t s = as_stream(stream);
+  const int nsm = num_sms_current();
+  int* status = at<int>(ws, L.status);
+  int32_t* topk_idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.topk_idx);
+  float* topk_gate = at<float>(ws, L.topk_gate);
+  int32_t* counts = expert_counts_out ? expert_counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_token = at<int32_t>(ws, L.row_token);
+  int32_t* row_map = at<int32_t>(ws, L.row_map);
+  const bool bf16 = dt == MOE_BF16;
+  // bf16 experts read A through TMA from the materialised x_perm; fp32 experts gather.
+  void* x_perm = bf16 ? at<void>(ws, L.x_perm) : nullptr;
+
+  auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], s) : cudaSuccess; };
+  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // 1. route (+ per-tile histogram)
+  if (mark(0) != cudaSuccess) return MOE_ERR_CUDA;
+  RouteArgs ra{};
+  ra.x = x; ra.wg = w_gate; ra.bias = gate_bias;
+  ra.T = T; ra.H = H; ra.E = E; ra.top_k = top_k; ra.dt_bf16 = bf16;
+  ra.topk_idx = topk_idx; ra.topk_gate = topk_gate; ra.logits_out = nullptr;
+  ra.tile_counts = at<int>(ws, L.tile_counts);
+  const RoutePlan rp = route_plan(T, H, E, bf16, nsm);
+  if (launch_route(ra, rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (mark(1) != cudaSuccess) return MOE_ERR_CUDA;
+  // 2. scan + scatter over the router's token tiles
+  PermuteArgs pa{};
+  pa.idx = topk_idx;
+  pa.T = T; pa.k = top_k; pa.E = E;
+  pa.BT = rp.BT; pa.tiles = rp.tiles;
+  pa.cap = capacity_of(capacity_factor, T, top_k, E);
+  pa.tile_counts = ra.tile_counts;
+  pa.counts = counts; pa.offsets = offsets; pa.row_token = row_token; pa.row_map = row_map;
+  pa.x = x; pa.x_perm = x_perm; pa.H = H; pa.elem_bytes = elem_bytes(dt);
+  pa.status = status;
+  if (launch_scan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (mark(2) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_scatter(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (mark(3) != cudaSuccess) return MOE_ERR_CUDA;
+  // 3. experts
+  const int R_max = T * top_k;
+  void* y = at<void>(ws, L.y);
+  st = run_ffn(x_perm, bf16 ? nullptr : row_token, x, w1, w3, w2, offsets, R_max, T, H, F, E, act,
+               dt, y, at<void>(ws, L.h), status, s, ev ? ev[4] : nullptr);
+  if (st != MOE_OK) return st;
+  if (mark(5) != cudaSuccess) return MOE_ERR_CUDA;
+  // 4. combine
+  if (launch_combine(y, topk_gate, row_map, T, H, top_k, bf16, out, nsm, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(mark(6));
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward(const void* x, const void* w_gate, const float* gate_bias, const void* w1,
+                       const void* w3, const void* w2, int T, int H, int F, int E, int top_k,
+                       float capacity_factor, moe_act act, moe_dtype dt, void* out,
+                       int32_t* topk_idx_out, int32_t* expert_counts_out, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(x, w_gate, gate_bias, w1, w3, w2, T, H, F, E, top_k, capacity_factor, act,
+                      dt, out, topk_idx_out, expert_counts_out, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_timed(const void* x, const void* w_gate, const float* gate_bias,
+                             const void* w1, const void* w3, const void* w2, int T, int H, int F,
+                             int E, int top_k, float capacity_factor, moe_act act, moe_dtype dt,
+                             void* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                             void* const* events, int n_events) {
+  if (!events || n_events < 7) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 7; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  return forward_impl(x, w_gate, gate_bias, w1, w3, w2, T, H, F, E, top_k, capacity_factor, act,
+                      dt, out, nullptr, nullptr, ws, ws_bytes, stream,
+                      reinterpret_cast<cudaEvent_t const*>(events));
+}
+
+moe_status moe_forward_host(const void* x_host, const void* w_gate, const float* gate_bias,
+                            const void* w1, const void* w3, const void* w2, int T, int H, int F,
+                            int E, int top_k, float capacity_factor, moe_act act, moe_dtype dt,
+                            void* out_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (F <= 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host || !ws) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, true);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const size_t bytes = static_cast<size_t>(T) * H * elem_bytes(dt);
+  void* xd = at<void>(ws, L.x_stage);
+  void* od = at<void>(ws, L.out_stage);
+  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = moe_forward(xd, w_gate, gate_bias, w1, w3, w2, T, H, F, E, top_k, capacity_factor, act, dt,
+                   od, nullptr, nullptr, ws, L.x_stage, stream);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+moe_status moe_get_device_status(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  switch (v) {
+    case 0: return MOE_OK;
+    case MOE_ERR_INVALID_ARG: return MOE_ERR_INVALID_ARG;
+    case MOE_ERR_INDEX_OUT_OF_RANGE: return MOE_ERR_INDEX_OUT_OF_RANGE;
+    case MOE_ERR_TIMEOUT: return MOE_ERR_TIMEOUT;
+    default: return MOE_ERR_CUDA;
+  }
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_INDEX_OUT_OF_RANGE: return "MOE_ERR_INDEX_OUT_OF_RANGE";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
+
+}  // extern "C"

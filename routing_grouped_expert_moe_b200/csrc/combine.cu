@@ -1,0 +1,94 @@
+// Deterministic weighted combine back to token order.
+//
+// "MoE模型高效推理：CANN算子库优化实践" §2.1 (the layer output is the sum of the
+// gate-weighted expert outputs); "ops-transformer 仓库 - MoE 算子优化实战"
+// (SparseScatterAdd); lshu.cn torch_npu article §4 (npu_moe_token_postprocess
+// restores token order).  The pages aggregate with atomic adds (hnwysp.cn
+// article §2.2, stage 3); here each token reads its own k rows and sums them in
+// slot order, so the result is the same bit for bit on every run.
+//
+// One warp per token, 16-byte vector loads of each kept row, fp32 accumulation
+// by FMA in slot order, one rounding to the storage type.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kCombineThreads = 256;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kCombineThreads)
+    k_combine(const uint8_t* __restrict__ y, const float* __restrict__ gate,
+              const int32_t* __restrict__ row_map, int T, int H, int k, uint8_t* __restrict__ out) {
+  constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
+  constexpr int EB = BF16 ? 2 : 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = H / EPV;
+  for (int t = blockIdx.x * (kCombineThreads / 32) + warp; t < T;
+       t += gridDim.x * (kCombineThreads / 32)) {
+    int rows[kMaxTopK];
+    float g[kMaxTopK];
+#pragma unroll
+    for (int s = 0; s < kMaxTopK; ++s) {
+      rows[s] = s < k ? __ldg(row_map + static_cast<size_t>(t) * k + s) : -1;
+      g[s] = s < k ? __ldg(gate + static_cast<size_t>(t) * k + s) : 0.f;
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[EPV];
+#pragma unroll
+      for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int s = 0; s < kMaxTopK; ++s) {
+        if (rows[s] < 0) continue;
+        const int4 q = __ldg(reinterpret_cast<const int4*>(
+            y + (static_cast<size_t>(rows[s]) * H + static_cast<size_t>(v) * EPV) * EB));
+        if constexpr (BF16) {
+          const uint32_t w[4] = {static_cast<uint32_t>(q.x), static_cast<uint32_t>(q.y),
+                                 static_cast<uint32_t>(q.z), static_cast<uint32_t>(q.w)};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(g[s], bf16_lo(w[i]), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(g[s], bf16_hi(w[i]), acc[2 * i + 1]);
+          }
+        } else {
+          acc[0] = fmaf(g[s], __int_as_float(q.x), acc[0]);
+          acc[1] = fmaf(g[s], __int_as_float(q.y), acc[1]);
+          acc[2] = fmaf(g[s], __int_as_float(q.z), acc[2]);
+          acc[3] = fmaf(g[s], __int_as_float(q.w), acc[3]);
+        }
+      }
+      int4 o;
+      if constexpr (BF16) {
+        o.x = static_cast<int>(pack_bf16x2(acc[0], acc[1]));
+        o.y = static_cast<int>(pack_bf16x2(acc[2], acc[3]));
+        o.z = static_cast<int>(pack_bf16x2(acc[4], acc[5]));
+        o.w = static_cast<int>(pack_bf16x2(acc[6], acc[7]));
+      } else {
+        o.x = __float_as_int(acc[0]);
+        o.y = __float_as_int(acc[1]);
+        o.z = __float_as_int(acc[2]);
+        o.w = __float_as_int(acc[3]);
+      }
+      *reinterpret_cast<int4*>(out + (static_cast<size_t>(t) * H + static_cast<size_t>(v) * EPV) *
+                                         EB) = o;
+    }
+  }
+}
+
+cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
+                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s) {
+  const int warps_per_cta = kCombineThreads / 32;
+  int grid = (T + warps_per_cta - 1) / warps_per_cta;
+  const int cap = num_sms * 8;  // resident CTAs; larger T loops inside the kernel
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  if (dt_bf16)
+    k_combine<true><<<grid, kCombineThreads, 0, s>>>(static_cast<const uint8_t*>(y), gate, row_map,
+                                                     T, H, k, static_cast<uint8_t*>(out));
+  else
+    k_combine<false><<<grid, kCombineThreads, 0, s>>>(static_cast<const uint8_t*>(y), gate,
+                                                      row_map, T, H, k, static_cast<uint8_t*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

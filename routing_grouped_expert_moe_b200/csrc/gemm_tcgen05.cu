@@ -1,0 +1,389 @@
+// Grouped expert GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// lshu.cn torch_npu fused-operator article §3 (x[tokens, hidden] times
+// expert_weight[num_experts, hidden, intermediate], then the activation and the
+// down-projection) and §4 (npu_moe_matmul); hnwysp.cn ops-transformer MoE
+// article §2.2 (the expert stage as one batched GEMM, fed by a prefetch stage,
+// aggregated by a reduce stage — here TMA producer, tcgen05 MMA and a TMEM
+// epilogue that runs concurrently with the next tile's main loop).
+//
+// One persistent CTA per SM walks a flat list of tiles (expert, n-tile, m-tile)
+// built on the device from expert_offsets, so the number of kept rows never
+// needs to reach the host.  m-tiles vary fastest, so the CTAs that share an
+// expert's weight tile run at the same time and the second read hits L2.
+//
+// Tile: 128 rows x 256 accumulator columns x 64 K per stage, 4 stages.
+//   A  (rows, K-major)       : 128 x 64 bf16, 128-byte swizzle, from a dense
+//                              row-major source (2-D TMA) or gathered row by row
+//                              through row_token (TMA tile::gather4).
+//   B  (weights, N-major)    : W[e] is [K, N] with N contiguous, so B is fed
+//                              MN-major: four 64-column TMA boxes, 128-byte swizzle.
+//   D  (TMEM, fp32)          : 2 x 256 columns (double-buffered accumulator).
+// Modes: 0 = gelu(A W1), 1 = silu(A W1) * (A W3) with W1 and W3 side by side in
+// one N=256 MMA (128 output columns), 2 = A W (down-projection).
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
+// owner), warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int G_BM = 128;
+constexpr int G_BK = 64;
+constexpr int G_STAGES = 4;
+constexpr int G_ACC_N = 256;
+constexpr int G_A_BYTES = G_BM * G_BK * 2;       // 16 KB
+constexpr int G_BCHUNK = 64 * G_BK * 2;          // one 64-column box: 8 KB
+constexpr int G_B_BYTES = G_ACC_N * G_BK * 2;    // 32 KB
+constexpr int G_STAGE_BYTES = G_A_BYTES + G_B_BYTES;
+constexpr int G_THREADS = 192;
+constexpr int G_SMEM = G_STAGES * G_STAGE_BYTES + 1024;
+constexpr uint32_t G_TMEM_COLS = 512;
+
+template <int MODE>
+struct ModeCfg {
+  static constexpr int BN_OUT = MODE == 1 ? 128 : 256;
+};
+
+struct TileInfo {
+  int e, m0, rows, n0;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int tau, const int* prefix, const int* seg_start,
+                                                const int* seg_rows, const int* mtiles, int E,
+                                                int bn_out) {
+  int lo = 0, hi = E;  // largest e with prefix[e] <= tau (empty experts are skipped)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= tau) lo = mid; else hi = mid;
+  }
+  TileInfo t;
+  t.e = lo;
+  const int local = tau - prefix[lo];
+  const int mt = mtiles[lo];
+  const int n_tile = local / mt;
+  const int m_tile = local - n_tile * mt;
+  t.m0 = seg_start[lo] + m_tile * G_BM;
+  t.rows = min(G_BM, seg_rows[lo] - m_tile * G_BM);
+  t.n0 = n_tile * bn_out;
+  return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ void epilogue_store(const float (&v)[32], const float (&u)[32],
+                                               __nv_bfloat16* dst, int cols_left) {
+  uint32_t p[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float a0 = v[2 * i], a1 = v[2 * i + 1];
+    if (MODE == 0) { a0 = gelu_f(a0); a1 = gelu_f(a1); }
+    if (MODE == 1) { a0 = silu_f(a0) * u[2 * i]; a1 = silu_f(a1) * u[2 * i + 1]; }
+    p[i] = pack_bf16x2(a0, a1);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (8 * j < cols_left) d[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+}
+
+template <int MODE, bool GATHER>
+__global__ void __launch_bounds__(G_THREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
+              const __grid_constant__ CUtensorMap tmB3, const GemmArgs args) {
+  constexpr int BN_OUT = ModeCfg<MODE>::BN_OUT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full_bar[G_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[G_STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int s_prefix[kMaxE + 1];
+  __shared__ int s_seg_start[kMaxE];
+  __shared__ int s_seg_rows[kMaxE];
+  __shared__ int s_mtiles[kMaxE];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  const int n_tiles_n = (args.N + BN_OUT - 1) / BN_OUT;
+  const int num_kb = (args.K + G_BK - 1) / G_BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < G_STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 128);
+    }
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    // Tile schedule from the expert segments: tiles(e) = ceil(rows_e/128) * n_tiles.
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      int rows = 0, s0 = 0;
+      if (e < E) {
+        s0 = args.offsets[e];
+        rows = args.offsets[e + 1] - s0;
+        if (rows < 0 || s0 < 0 || s0 + rows > args.R_max) {  // malformed segment: skip it
+          record_status(args.status, 1);
+          rows = 0;
+        }
+        s_seg_start[e] = s0;
+        s_seg_rows[e] = rows;
+      }
+      const int mt = (rows + G_BM - 1) / G_BM;
+      if (e < E) s_mtiles[e] = mt;
+      int v = mt * n_tiles_n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      if (e < E) s_prefix[e + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      s_prefix[0] = 0;
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB1);
+      if (MODE == 1) tma_prefetch_desc(&tmB3);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, G_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int total = s_prefix[E];
+  volatile int* abort_flag = &abort_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+      const TileInfo ti = decode_tile(tau, s_prefix, s_seg_start, s_seg_rows, s_mtiles, E, BN_OUT);
+      int r4[4] = {0, 0, 0, 0};
+      if (GATHER) {
+        const int first = args.row_token[ti.m0];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = lane * 4 + j;
+          r4[j] = i < ti.rows ? args.row_token[ti.m0 + i] : first;
+        }
+      }
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, args.status);
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        uint8_t* sA = smem + stage * G_STAGE_BYTES;
+        uint8_t* sB = sA + G_A_BYTES;
+        const int k0 = kb * G_BK;
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], G_STAGE_BYTES);
+        __syncwarp();
+        if (GATHER) {
+          tma_gather4(sA + lane * 512, &tmA, &full_bar[stage], k0, r4[0], r4[1], r4[2], r4[3]);
+        } else if (lane == 0) {
+          tma_load_2d(sA, &tmA, &full_bar[stage], k0, ti.m0);
+        }
+        if (lane == 0) {
+          if (MODE == 1) {
+            tma_load_3d(sB, &tmB1, &full_bar[stage], ti.n0, k0, ti.e);
+            tma_load_3d(sB + G_BCHUNK, &tmB1, &full_bar[stage], ti.n0 + 64, k0, ti.e);
+            tma_load_3d(sB + 2 * G_BCHUNK, &tmB3, &full_bar[stage], ti.n0, k0, ti.e);
+            tma_load_3d(sB + 3 * G_BCHUNK, &tmB3, &full_bar[stage], ti.n0 + 64, k0, ti.e);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_3d(sB + j * G_BCHUNK, &tmB1, &full_bar[stage], ti.n0 + 64 * j, k0, ti.e);
+          }
+        }
+        if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(G_BM, G_ACC_N, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * G_ACC_N);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * G_STAGE_BYTES);
+          const uint32_t b_base = a_base + G_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < G_BK / 16; ++kk) {
+            // A: K-major, rows of 128 B, 8-row groups 1024 B apart; K step = 32 B.
+            const uint64_t adesc = smem_desc(a_base + kk * 32, 16, 1024);
+            // B: MN-major, 64-column boxes 8 KB apart (LBO), 8 K-rows 1024 B apart (SBO);
+            //    K step of 16 rows = 2048 B.
+            const uint64_t bdesc = smem_desc(b_base + kk * 2048, G_BCHUNK, 1024);
+            umma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == G_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const int row = q * 32 + lane;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
+      const TileInfo ti = decode_tile(tau, s_prefix, s_seg_start, s_seg_rows, s_mtiles, E, BN_OUT);
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, args.status);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      tc_fence_after();
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * G_ACC_N);
+      const bool row_ok = row < ti.rows;
+      __nv_bfloat16* orow =
+          row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
+      if (MODE == 1) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float g[32], u[32];
+          tmem_ld32(t_row + c * 32, g);
+          tmem_ld32(t_row + 128 + c * 32, u);
+          tmem_ld_wait();
+          const int cols_left = args.N - (ti.n0 + c * 32);
+          if (row_ok && cols_left > 0) epilogue_store<1>(g, u, orow + c * 32, cols_left);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float v[32];
+          tmem_ld32(t_row + c * 32, v);
+          tmem_ld_wait();
+          const int cols_left = args.N - (ti.n0 + c * 32);
+          if (row_ok && cols_left > 0) epilogue_store<MODE>(v, v, orow + c * 32, cols_left);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, G_TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host: tensor maps and launch
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows, cols] (cols contiguous) with box {64, box_rows}, 128-byte swizzle.
+static bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over W[E, K, N] (N contiguous), box {64 N, 64 K, 1}, 128-byte swizzle.
+static bool make_map_w(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {N, K, E};
+  cuuint64_t strides[2] = {N * 2, K * N * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, bool GATHER>
+static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const CUtensorMap& b3,
+                             const GemmArgs& g, int num_sms, cudaStream_t s) {
+  auto kern = k_gemm_tc<MODE, GATHER>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
+    if (err != cudaSuccess) return err;
+    attr_set = true;
+  }
+  kern<<<num_sms, G_THREADS, G_SMEM, s>>>(a, b1, b3, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
+                           const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s) {
+  CUtensorMap ma, mb1, mb3;
+  // A: [a_rows, K]; dense source uses 128-row boxes, the gathered source 1-row boxes.
+  if (!make_map_2d(&ma, a_src, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(g.K),
+                   gather ? 1u : static_cast<uint32_t>(G_BM)))
+    return cudaErrorInvalidValue;
+  if (!make_map_w(&mb1, b1, g.E, g.K, g.N)) return cudaErrorInvalidValue;
+  if (mode == 1) {
+    if (!make_map_w(&mb3, b3, g.E, g.K, g.N)) return cudaErrorInvalidValue;
+  } else {
+    mb3 = mb1;
+  }
+  switch (mode * 2 + (gather ? 1 : 0)) {
+    case 0: return launch_tc<0, false>(ma, mb1, mb3, g, num_sms, s);
+    case 1: return launch_tc<0, true>(ma, mb1, mb3, g, num_sms, s);
+    case 2: return launch_tc<1, false>(ma, mb1, mb3, g, num_sms, s);
+    case 3: return launch_tc<1, true>(ma, mb1, mb3, g, num_sms, s);
+    case 4: return launch_tc<2, false>(ma, mb1, mb3, g, num_sms, s);
+    case 5: return launch_tc<2, true>(ma, mb1, mb3, g, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,94 @@
+// Internal launch interfaces between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxTopK = 8;
+
+// ---------------------------------------------------------------- router
+struct RouteArgs {
+  const void* x;        // [T,H] bf16 or fp32
+  const void* wg;       // [H,E]
+  const float* bias;    // [E] or null
+  int T, H, E, top_k, dt_bf16;
+  int32_t* topk_idx;    // [T,k]
+  float* topk_gate;     // [T,k]
+  float* logits_out;    // [T,E] or null
+  int* tile_counts;     // [tiles,E] or null: per-tile expert histogram
+};
+
+struct RoutePlan {
+  int kind;   // 0 = SIMT, 1 = tensor-core (mma.sync) path
+  int MT;     // 16-token m-tiles per CTA (tensor-core path)
+  int NTP;    // 8-expert n-tiles, rounded up to a power of two
+  int BT;     // tokens per CTA tile
+  int tiles;  // CTA tiles along T
+  int ck;     // CTAs per cluster splitting H
+};
+
+RoutePlan route_plan(int T, int H, int E, int dt_bf16, int num_sms);
+cudaError_t launch_route(const RouteArgs& a, const RoutePlan& p, cudaStream_t s);
+cudaError_t launch_route_from_logits(const RouteArgs& a, const float* logits, cudaStream_t s);
+
+// ---------------------------------------------------------------- permute
+struct PermuteArgs {
+  const int32_t* idx;   // [T,k] expert ids
+  int T, k, E;
+  int BT;               // tokens per tile (must match the histogram's tiling)
+  int tiles;
+  int cap;              // per-expert capacity (INT32_MAX when unlimited)
+  int* tile_counts;     // [tiles,E] histogram in, tile bases out (in place)
+  int32_t* counts;      // [E]   pre-drop counts
+  int32_t* offsets;     // [E+1] post-drop exclusive prefix
+  int32_t* row_token;   // [T*k]
+  int32_t* row_map;     // [T*k]
+  const void* x;        // [T,H] (for x_perm) or null
+  void* x_perm;         // [T*k,H] or null
+  int H, elem_bytes;
+  int* status;
+};
+
+constexpr int kPermuteBT = 128;
+cudaError_t launch_hist(const PermuteArgs& a, cudaStream_t s);
+cudaError_t launch_scan(const PermuteArgs& a, cudaStream_t s);
+cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- grouped GEMM
+// MODE 0: out = gelu(A B1); MODE 1: out = silu(A B1) * (A B3); MODE 2: out = A B1.
+struct GemmArgs {
+  const int32_t* offsets;    // [E+1] row segments per expert
+  const int32_t* row_token;  // gathered A rows (GATHER) or null
+  int E, N, K;               // output columns, reduction length
+  int R_max;                 // rows available in the output / row_token
+  int T;                     // rows of the gathered source
+  void* out;                 // [R_max, N]
+  int* status;
+};
+
+struct GemmTcPlan {
+  CUtensorMap tmA, tmB1, tmB3;
+};
+
+// bf16 tensor-core (tcgen05) path. a_src: x_perm/h rows (dense) or x (gather).
+cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
+                           const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s);
+// fp32 CUDA-core path (no TF32).
+cudaError_t launch_gemm_simt(int mode, const void* a_src, const void* b1, const void* b3,
+                             const GemmArgs& g, int num_sms, cudaStream_t s);
+// Identity experts: out[r] = a[r] or x[row_token[r]].
+cudaError_t launch_copy_rows(const void* a_src, const GemmArgs& g, int elem_bytes,
+                             cudaStream_t s);
+
+// ---------------------------------------------------------------- combine
+cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
+                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- misc
+cudaError_t launch_clear_status(int* status, cudaStream_t s);
+
+}  // namespace moe

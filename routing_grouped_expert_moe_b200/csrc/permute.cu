@@ -1,0 +1,197 @@
+// Permute / dispatch: expert histogram, capacity clamp + offsets, and the
+// stable scatter that gives every kept (token, slot) pair its expert-major row.
+//
+// lshu.cn torch_npu fused-operator article §4 (npu_moe_token_preprocess: token
+// rearrangement), §5.2 (expert ids are int32 in [0, num_experts) — out-of-range
+// ids are errors, never clamped), §5.3 (a fixed-size buffer per expert, which a
+// skewed router overflows); hnwysp.cn ops-transformer MoE article §3.2
+// (capacity_factor); "ops-transformer 仓库 - MoE 算子优化实战" (SparseGather,
+// CSR storage of the sparse assignment).
+//
+// Pairs are ordered by a = t*k + s.  The tokens are cut into tiles of BT; the
+// histogram gives per-tile counts, one CTA scans them per expert (tile bases,
+// pre-drop counts, capacity clamp, offsets), and the scatter recomputes each
+// pair's rank inside its tile with warp match/popc, so rank = tile base + rank
+// in tile is the pair's arrival order among all pairs of that expert.
+#include <climits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kPermThreads = 256;
+
+// Per-tile expert histogram of caller-given ids (the fused path gets it from
+// the router).  Out-of-range ids are reported and not counted.
+__global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
+  __shared__ int cnt_s[kMaxE];
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < a.E; i += kPermThreads) cnt_s[i] = 0;
+  __syncthreads();
+  const int a0 = blockIdx.x * a.BT * a.k;
+  const int a1 = min(a.T, (blockIdx.x + 1) * a.BT) * a.k;
+  for (int base = a0; base < a1; base += kPermThreads) {
+    const int i = base + threadIdx.x;
+    int e = -1;
+    if (i < a1) {
+      e = a.idx[i];
+      if (e < 0 || e >= a.E) {
+        record_status(a.status, kStatusIndexOutOfRange);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt_s[e], __popc(peers));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.E; i += kPermThreads)
+    a.tile_counts[static_cast<size_t>(blockIdx.x) * a.E + i] = cnt_s[i];
+}
+
+// One CTA: per-expert exclusive scan over tiles (written back in place as
+// tile bases), pre-drop counts, kept = min(count, C), offsets = scan(kept).
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) k_scan(PermuteArgs a) {
+  __shared__ int buf[kScanThreads];
+  __shared__ int carry[kMaxE];
+  int Ep = 1;
+  while (Ep < a.E) Ep <<= 1;
+  const int P = kScanThreads / Ep;  // tiles handled per round
+  const int e = threadIdx.x % Ep, p = threadIdx.x / Ep;
+  for (int i = threadIdx.x; i < a.E; i += kScanThreads) carry[i] = 0;
+  __syncthreads();
+  for (int base = 0; base < a.tiles; base += P) {
+    const int j = base + p;
+    const bool ok = (e < a.E) && (j < a.tiles);
+    const int v = ok ? a.tile_counts[static_cast<size_t>(j) * a.E + e] : 0;
+    buf[threadIdx.x] = v;
+    __syncthreads();
+    for (int off = 1; off < P; off <<= 1) {
+      const int u = (p >= off) ? buf[threadIdx.x - off * Ep] : 0;
+      __syncthreads();
+      buf[threadIdx.x] += u;
+      __syncthreads();
+    }
+    if (ok) a.tile_counts[static_cast<size_t>(j) * a.E + e] = carry[e] + buf[threadIdx.x] - v;
+    __syncthreads();
+    if (p == P - 1 && e < a.E) carry[e] += buf[threadIdx.x];
+    __syncthreads();
+  }
+  if (threadIdx.x < 32) {
+    int run = 0;
+    for (int b = 0; b < a.E; b += 32) {
+      const int ee = b + threadIdx.x;
+      int kept = 0;
+      if (ee < a.E) {
+        a.counts[ee] = carry[ee];
+        kept = min(carry[ee], a.cap);
+      }
+      int incl = kept;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (threadIdx.x >= off) incl += u;
+      }
+      if (ee < a.E) a.offsets[ee] = run + incl - kept;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (threadIdx.x == 0) a.offsets[a.E] = run;
+  }
+}
+
+// Stable scatter.  CTA j handles pairs [j*BT*k, min(T,(j+1)*BT)*k) in rounds
+// of 256; inside a round a pair's rank among same-expert pairs comes from
+// __match_any_sync (rank in warp) plus an exclusive scan over warps.
+constexpr int kScatterMaxPairs = 128 * kMaxTopK;
+
+__global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
+  __shared__ int wcnt[kPermThreads / 32][kMaxE];
+  __shared__ int running[kMaxE];
+  __shared__ int rows_s[kScatterMaxPairs];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x;
+  const int a0 = j * a.BT * a.k;
+  const int a1 = min(a.T, (j + 1) * a.BT) * a.k;
+  for (int i = threadIdx.x; i < a.E; i += kPermThreads) running[i] = 0;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = a0; base < a1; base += kPermThreads) {
+    for (int i = threadIdx.x; i < (kPermThreads / 32) * a.E; i += kPermThreads)
+      wcnt[i / a.E][i % a.E] = 0;
+    __syncthreads();
+    const int i = base + threadIdx.x;
+    int e = -1;
+    if (i < a1) {
+      e = a.idx[i];
+      if (e < 0 || e >= a.E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & lt_mask);
+    if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < a.E; ee += kPermThreads) {
+      int s = running[ee];
+#pragma unroll
+      for (int w = 0; w < kPermThreads / 32; ++w) {
+        const int c = wcnt[w][ee];
+        wcnt[w][ee] = s;
+        s += c;
+      }
+      running[ee] = s;
+    }
+    __syncthreads();
+    if (i < a1) {
+      int row = -1;
+      if (e >= 0) {
+        const int rank = a.tile_counts[static_cast<size_t>(j) * a.E + e] + wcnt[warp][e] + rank_w;
+        if (rank < a.cap) {
+          row = a.offsets[e] + rank;
+          a.row_token[row] = i / a.k;
+        }
+      }
+      a.row_map[i] = row;
+      rows_s[i - a0] = row;
+    }
+    __syncthreads();
+  }
+  if (a.x_perm == nullptr) return;
+  // Gather the kept rows of x into x_perm: one warp per pair, 16-byte vectors.
+  const int row_bytes = a.H * a.elem_bytes;
+  const int vecs = row_bytes / 16;
+  for (int p = a0 + warp; p < a1; p += kPermThreads / 32) {
+    const int row = rows_s[p - a0];
+    if (row < 0) continue;
+    const int t = p / a.k;
+    const int4* src = reinterpret_cast<const int4*>(static_cast<const uint8_t*>(a.x) +
+                                                    static_cast<size_t>(t) * row_bytes);
+    int4* dst = reinterpret_cast<int4*>(static_cast<uint8_t*>(a.x_perm) +
+                                        static_cast<size_t>(row) * row_bytes);
+    for (int v = lane; v < vecs; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+cudaError_t launch_hist(const PermuteArgs& a, cudaStream_t s) {
+  k_hist<<<a.tiles, kPermThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const PermuteArgs& a, cudaStream_t s) {
+  k_scan<<<1, kScanThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s) {
+  if (a.BT * a.k > kScatterMaxPairs) return cudaErrorInvalidValue;
+  k_scatter<<<a.tiles, kPermThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+__global__ void k_clear_status(int* status) { *status = 0; }
+
+cudaError_t launch_clear_status(int* status, cudaStream_t s) {
+  k_clear_status<<<1, 1, 0, s>>>(status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

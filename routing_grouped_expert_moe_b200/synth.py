@@ -27,6 +27,7 @@ Workloads (the shapes of the pages' own examples):
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -103,24 +104,40 @@ NUMBERED = ["tiny_f32", "page1_gelu", "mixtral_e8", "e32_long", "e128_skew"]
 UNIFORM_BIAS = 0.5
 
 
-def _generator(seed: int, stream: int, attempt: int = 0) -> np.random.Generator:
-    ss = np.random.SeedSequence([seed, stream, attempt])
+def _generator(seed: int, stream: int, attempt: int = 0, chunk: int = 0) -> np.random.Generator:
+    ss = np.random.SeedSequence([seed, stream, attempt, chunk])
     return np.random.Generator(np.random.Philox(ss))
+
+
+_CHUNK = 1 << 24
 
 
 def normal(seed: int, stream: int, shape, std: float, dtype: torch.dtype,
            attempt: int = 0) -> torch.Tensor:
-    """N(0, std^2) draws from one Philox stream, stored (round-to-nearest-even) in dtype."""
-    g = _generator(seed, stream, attempt)
+    """N(0, std^2) draws stored (round-to-nearest-even) in dtype.
+
+    Element i comes from Philox sub-stream (seed, stream, attempt, i // 2**24),
+    so chunks are drawn in parallel and the result does not depend on threads.
+    """
+    from concurrent.futures import ThreadPoolExecutor
     n = int(np.prod(shape))
     out = torch.empty(n, dtype=dtype)
-    chunk = 1 << 26
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        a = g.standard_normal(e - s, dtype=np.float32)
+
+    def fill(ci):
+        s = ci * _CHUNK
+        e = min(n, s + _CHUNK)
+        a = _generator(seed, stream, attempt, ci).standard_normal(e - s, dtype=np.float32)
         if std != 1.0:
             a *= np.float32(std)
         out[s:e] = torch.from_numpy(a).to(dtype)
+
+    nchunks = (n + _CHUNK - 1) // _CHUNK
+    if nchunks <= 1:
+        for ci in range(nchunks):
+            fill(ci)
+    else:
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(nchunks)))
     return out.view(*shape)
 
 

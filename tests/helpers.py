@@ -1,0 +1,61 @@
+"""Test-side helpers: gap-enforced workload inputs and error metrics.
+
+The router-logit gap rule (every consecutive gap among a token's top k+1
+logits >= 1e-3, so selection has no near-ties) needs the layer's own logits;
+it therefore lives here, on the test side, and uses the oracle's logits.
+Violating tokens' x rows are redrawn from the generator's redraw stream.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import moe_oracle as O
+from routing_grouped_expert_moe_b200 import synth
+
+MIN_GAP = 1e-3
+TOL = {"f32": 1e-4, "bf16": 2e-2}   # max|gpu - oracle| / max|oracle|
+
+
+def as_np(t: torch.Tensor) -> np.ndarray:
+    """Exact float64 (or int) numpy copy of a CPU/GPU tensor."""
+    t = t.detach().cpu()
+    if t.is_floating_point():
+        return t.to(torch.float64).numpy()
+    return t.numpy()
+
+
+def gap_violations(logits: np.ndarray, k: int, min_gap: float = MIN_GAP) -> np.ndarray:
+    E = logits.shape[1]
+    m = min(k + 1, E)
+    srt = -np.sort(-logits.astype(np.float64), axis=1)[:, :m]
+    gaps = srt[:, :-1] - srt[:, 1:]
+    return np.nonzero(np.any(gaps < min_gap, axis=1))[0]
+
+
+def gapped_inputs(cfg: synth.MoEConfig, with_weights: bool = True, max_rounds: int = 50) -> dict:
+    d = synth.make_inputs(cfg, with_weights=with_weights)
+    x = d["x"]
+    wg = as_np(d["w_gate"])
+    b = None if d["gate_bias"] is None else as_np(d["gate_bias"])
+    bad = np.arange(cfg.T)
+    for attempt in range(max_rounds):
+        lg = O.router_logits(as_np(x[torch.from_numpy(bad)]) if attempt else as_np(x), wg, b)
+        viol = gap_violations(lg, cfg.top_k)
+        bad = bad[viol] if attempt else viol
+        if len(bad) == 0:
+            break
+        x[torch.from_numpy(bad)] = synth.redraw_rows(cfg, len(bad), attempt)
+    else:
+        raise RuntimeError("gap enforcement did not converge")
+    d["x"] = x
+    return d
+
+
+def rel_err(gpu, ref) -> float:
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    denom = np.max(np.abs(r)) if r.size else 0.0
+    if denom == 0.0:
+        return float(np.max(np.abs(g))) if g.size else 0.0
+    return float(np.max(np.abs(g - r)) / denom)

@@ -1,0 +1,142 @@
+"""Whole-layer parity of moe_forward (the call bench.py times) against the oracle.
+
+Small workloads are compared on every output element.  The full-size
+workloads run in exactly the launch configuration the bench times; the oracle
+recomputes routing for every token (indices and pre-drop counts must match bit
+for bit) and the expert FFN + combine for a sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from routing_grouped_expert_moe_b200 import synth
+from tests.helpers import TOL, as_np, gapped_inputs, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def B():
+    from routing_grouped_expert_moe_b200 import binding
+    return binding
+
+
+def _cuda(d):
+    return {k: (None if v is None else v.cuda()) for k, v in d.items()}
+
+
+def _run(cfg, d, act=None):
+    g = _cuda(d)
+    T, E, k = cfg.T, cfg.E, cfg.top_k
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(E, dtype=torch.int32, device="cuda")
+    ws = B().alloc_workspace(B().workspace_bytes(T, cfg.H, cfg.F, E, k, act or cfg.act,
+                                                 cfg.torch_dtype))
+    out = B().forward(g["x"], g["w_gate"], g["gate_bias"], g.get("w1"), g.get("w3"), g.get("w2"),
+                      k, cfg.capacity_factor, act or cfg.act, ws=ws, topk_idx_out=idx,
+                      expert_counts_out=cnt)
+    assert B().device_status(ws) == B().OK
+    return out, idx, cnt, ws
+
+
+def _small_cfg(base_name, **kw):
+    base = synth.CONFIGS[base_name]
+    from dataclasses import replace
+    return replace(base, **kw)
+
+
+SMALL = [
+    synth.CONFIGS["tiny_f32"],
+    synth.CONFIGS["drop_cf05"],
+    _small_cfg("page1_gelu", name="gelu_small", T=700, H=256, F=512, seed=2001),
+    _small_cfg("mixtral_e8", name="swiglu_small", T=333, H=512, F=384, seed=2002),
+    _small_cfg("e128_skew", name="skew_small", T=1500, H=256, F=128, seed=2003),
+    _small_cfg("e32_long", name="e32_small", T=2049, H=128, F=1376, capacity_factor=1.0,
+               seed=2004),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_forward_small_full_compare(cfg):
+    d = gapped_inputs(cfg)
+    out, idx, cnt, _ = _run(cfg, d)
+    ref = O.moe_forward(as_np(d["x"]), as_np(d["w_gate"]),
+                        None if d["gate_bias"] is None else as_np(d["gate_bias"]),
+                        as_np(d["w1"]), None if d["w3"] is None else as_np(d["w3"]),
+                        as_np(d["w2"]), cfg.top_k, cfg.capacity_factor, cfg.act, cfg.dtype)
+    np.testing.assert_array_equal(as_np(idx), ref["topk_idx"])
+    np.testing.assert_array_equal(as_np(cnt), ref["counts"])
+    err = rel_err(as_np(out), ref["out"])
+    assert err <= TOL[cfg.dtype], err
+    if cfg.name == "drop_cf05":
+        assert ref["dropped"] > 0
+
+
+@pytest.mark.parametrize("name", ["page1_gelu", "mixtral_e8", "e32_long", "e128_skew"])
+def test_forward_full_size_sampled(name):
+    cfg = synth.CONFIGS[name]
+    d = gapped_inputs(cfg)
+    out, idx, cnt, _ = _run(cfg, d)
+    x = as_np(d["x"]).astype(np.float32)
+    lg = O.router_logits(x, as_np(d["w_gate"]),
+                         None if d["gate_bias"] is None else as_np(d["gate_bias"]))
+    rng = np.random.default_rng(cfg.seed)
+    toks = np.unique(np.concatenate([[0, 1, cfg.T - 1], rng.choice(cfg.T, 45, replace=False)]))
+    w = {k: (None if d[k] is None else d[k].float().numpy()) for k in ("w1", "w3", "w2")}
+    ref = O.moe_forward_sampled(x, lg, w["w1"], w["w3"], w["w2"], cfg.top_k,
+                                cfg.capacity_factor, cfg.act, cfg.dtype, toks)
+    np.testing.assert_array_equal(as_np(idx), ref["topk_idx"])
+    np.testing.assert_array_equal(as_np(cnt), ref["counts"])
+    err = rel_err(as_np(out)[toks], ref["out_rows"])
+    assert err <= TOL[cfg.dtype], err
+
+
+def test_forward_identity_experts_give_x_times_gate_sum():
+    cfg = _small_cfg("drop_cf05", name="identity", T=900, H=128, F=8)
+    d = gapped_inputs(cfg, with_weights=False)
+    out, idx, cnt, _ = _run(cfg, {**d, "w1": None, "w3": None, "w2": None}, act="identity")
+    lg = O.router_logits(as_np(d["x"]), as_np(d["w_gate"]), None)
+    ref = O.moe_forward(as_np(d["x"]), None, None, None, None, None, cfg.top_k,
+                        cfg.capacity_factor, "identity", cfg.dtype, logits=lg)
+    assert ref["dropped"] > 0
+    g = ref["topk_gate"].astype(np.float64) * (ref["row_map"] >= 0)
+    np.testing.assert_allclose(as_np(out), as_np(d["x"]) * g.sum(1, keepdims=True), rtol=8e-3,
+                               atol=1e-2)
+    assert rel_err(as_np(out), ref["out"]) <= TOL["bf16"]
+
+
+def test_forward_single_expert_is_dense_ffn():
+    cfg = _small_cfg("mixtral_e8", name="dense", T=300, H=256, F=512, E=1, top_k=1, seed=2010)
+    d = synth.make_inputs(cfg)
+    out, *_ = _run(cfg, d)
+    xt = d["x"].double()
+    h = torch.nn.functional.silu(xt @ d["w1"][0].double()) * (xt @ d["w3"][0].double())
+    ref = h.to(torch.bfloat16).double() @ d["w2"][0].double()
+    assert rel_err(as_np(out), ref.numpy()) <= TOL["bf16"]
+
+
+def test_forward_deterministic_and_host_entry_point():
+    cfg = _small_cfg("page1_gelu", name="det", T=1024, H=512, F=1024, seed=2020)
+    d = synth.make_inputs(cfg)
+    o1, *_ = _run(cfg, d)
+    o2, *_ = _run(cfg, d)
+    assert torch.equal(o1, o2)
+    g = _cuda(d)
+    xh = d["x"].pin_memory()
+    oh = B().forward_host(xh, g["w_gate"], g["gate_bias"], g["w1"], None, g["w2"], cfg.top_k,
+                          cfg.capacity_factor, cfg.act)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o1.cpu())
+
+
+def test_forward_empty_and_one_token():
+    cfg = _small_cfg("mixtral_e8", name="one", T=1, H=256, F=256, seed=2030)
+    d = synth.make_inputs(cfg)
+    out, idx, cnt, _ = _run(cfg, d)
+    ref = O.moe_forward(as_np(d["x"]), as_np(d["w_gate"]), None, as_np(d["w1"]), as_np(d["w3"]),
+                        as_np(d["w2"]), cfg.top_k, 0.0, cfg.act, cfg.dtype)
+    assert rel_err(as_np(out), ref["out"]) <= TOL["bf16"]
+    g = _cuda(d)
+    empty = torch.empty(0, cfg.H, dtype=torch.bfloat16, device="cuda")
+    o = B().forward(empty, g["w_gate"], None, g["w1"], g["w3"], g["w2"], 2, 0.0, "swiglu")
+    assert o.shape == (0, cfg.H)

@@ -1,0 +1,191 @@
+"""Per-stage parity of the CUDA path against the oracle, through the C ABI.
+
+Integer outputs (expert ids, counts, offsets, row maps) must match bit for bit;
+floating point outputs within max|gpu - oracle| / max|oracle| <= 1e-4 (fp32) or
+2e-2 (bf16).  Sizes span several tiles and a ragged tail.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from routing_grouped_expert_moe_b200 import synth
+from tests.helpers import TOL, as_np, gap_violations, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def B():
+    from routing_grouped_expert_moe_b200 import binding
+    return binding
+
+
+# ---------------------------------------------------------------- router
+
+@pytest.mark.parametrize("T,E,k", [(1, 4, 1), (37, 8, 2), (300, 32, 2), (1000, 128, 2),
+                                   (129, 256, 8), (77, 5, 5), (64, 12, 3)])
+def test_route_from_logits_bit_exact(T, E, k):
+    lg = synth.random_logits(100 + T, T, E, scale=2.0)
+    lg[0, :] = 0.5                         # a token of all-equal logits: lower ids win
+    if T > 2:
+        lg[1, 0] = float("nan")
+        lg[2, E - 1] = float("-inf")
+    idx, gate = B().route_from_logits(lg.cuda(), k)
+    ref_idx = O.topk_select(lg.numpy(), k)
+    np.testing.assert_array_equal(as_np(idx), ref_idx)
+    ok = np.isfinite(lg.numpy()).all(axis=1)
+    ref_g = O.topk_gates(lg.numpy(), ref_idx)
+    np.testing.assert_allclose(as_np(gate)[ok], ref_g[ok], rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("dtype,T,H,E,k", [
+    ("bf16", 1000, 512, 8, 2), ("bf16", 333, 1024, 32, 2), ("bf16", 517, 256, 128, 2),
+    ("bf16", 64, 4096, 8, 2),                       # few tiles: H split over a cluster
+    ("bf16", 96, 200, 16, 4),                       # H not a multiple of the 128 chunk
+    ("bf16", 50, 64, 12, 3),                        # E not a multiple of 8 (CUDA-core path)
+    ("f32", 257, 128, 4, 2), ("f32", 100, 96, 40, 3),
+])
+def test_route_from_x(dtype, T, H, E, k):
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = synth.normal(7, 0, (T, H), 1.0, dt)
+    wg = synth.normal(7, 1, (H, E), H ** -0.5, dt)
+    bias = synth.normal(7, 2, (E,), 0.1, torch.float32)
+    idx, gate, lg = B().route(x.cuda(), wg.cuda(), bias.cuda(), top_k=k, logits_out=True)
+    ref_lg = O.router_logits(as_np(x), as_np(wg), as_np(bias))
+    # logits: fp32 accumulation in a different order than the float64 oracle
+    assert rel_err(as_np(lg), ref_lg) < 1e-5
+    # selection from the GPU's own logits follows the selection rule exactly
+    np.testing.assert_array_equal(as_np(idx), O.topk_select(as_np(lg).astype(np.float32), k))
+    # and agrees with the oracle's selection wherever the top-k gaps are clear
+    clear = np.setdiff1d(np.arange(T), gap_violations(ref_lg, k))
+    np.testing.assert_array_equal(as_np(idx)[clear], O.topk_select(ref_lg, k)[clear])
+    np.testing.assert_allclose(as_np(gate)[clear],
+                               O.topk_gates(ref_lg, O.topk_select(ref_lg, k))[clear],
+                               rtol=1e-4, atol=1e-6)
+
+
+# ---------------------------------------------------------------- permute
+
+def _perm_check(ids, E, cf, x=None):
+    r = B().permute(ids.cuda(), E, capacity_factor=cf, x=None if x is None else x.cuda())
+    cap = O.capacity(cf, ids.shape[0], ids.shape[1], E)
+    ref = O.permute(ids.numpy(), E, cap)
+    np.testing.assert_array_equal(as_np(r["counts"]), ref["counts"])
+    np.testing.assert_array_equal(as_np(r["offsets"]), ref["offsets"])
+    R = ref["R"]
+    np.testing.assert_array_equal(as_np(r["row_token"])[:R], ref["row_token"])
+    np.testing.assert_array_equal(as_np(r["row_map"]), ref["row_map"])
+    assert B().device_status(r["ws"]) == B().OK
+    if x is not None:
+        np.testing.assert_array_equal(as_np(r["x_perm"])[:R], as_np(x)[ref["row_token"]])
+    return r, ref
+
+
+@pytest.mark.parametrize("T,E,k,cf,skew", [
+    (1, 4, 2, 0.0, 0.0), (1000, 8, 2, 0.0, 0.0), (4097, 32, 2, 1.25, 0.0),
+    (3000, 128, 2, 0.0, 0.05), (777, 8, 2, 0.5, 0.3), (2000, 16, 4, 1.0, 0.2),
+    (513, 256, 8, 0.0, 0.0), (300, 3, 1, 0.8, 1.0),
+])
+def test_permute_bit_exact(T, E, k, cf, skew):
+    ids = synth.random_expert_ids(T + E, T, E, k, skew=skew)
+    x = synth.normal(3, 0, (T, 64), 1.0, torch.bfloat16)
+    _perm_check(ids, E, cf, x)
+
+
+def test_permute_golden_cases():
+    import json, os
+    here = os.path.join(os.path.dirname(__file__), "golden", "capacity_cases.json")
+    for c in json.load(open(here))["cases"]:
+        ids = torch.tensor(c["topk_idx"], dtype=torch.int32)
+        r, _ = _perm_check(ids, c["E"], c["capacity_factor"])
+        np.testing.assert_array_equal(as_np(r["row_map"]), np.array(c["row_map"]))
+
+
+def test_permute_all_to_one_expert_with_capacity():
+    T, E, k = 5000, 8, 2
+    ids = torch.stack([torch.zeros(T, dtype=torch.int32), torch.ones(T, dtype=torch.int32)], 1)
+    _perm_check(ids, E, 1.0)                         # C = 1250: 3750 pairs dropped per expert
+
+
+def test_permute_out_of_range_is_reported():
+    ids = synth.random_expert_ids(1, 300, 8, 2)
+    ids[17, 1] = 8
+    ids[200, 0] = -3
+    r = B().permute(ids.cuda(), 8)
+    assert B().device_status(r["ws"]) == B().ERR_INDEX_OUT_OF_RANGE
+    rm = as_np(r["row_map"])
+    assert rm[17, 1] == -1 and rm[200, 0] == -1
+    assert as_np(r["counts"]).sum() == 300 * 2 - 2
+    assert B().device_status(r["ws"]) == B().OK      # reading clears it
+
+
+# ---------------------------------------------------------------- grouped FFN
+
+def _ffn_case(dtype, act, E, rows_per_expert, H, F, seed=11):
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    T = max(1, sum(rows_per_expert))
+    x = synth.normal(seed, 0, (T, H), 1.0, dt)
+    w1 = synth.normal(seed, 2, (E, H, F), H ** -0.5, dt)
+    w3 = synth.normal(seed, 3, (E, H, F), H ** -0.5, dt) if act == "swiglu" else None
+    w2 = synth.normal(seed, 4, (E, F, H), F ** -0.5, dt)
+    # a k=1 assignment with the requested rows per expert, tokens shuffled
+    ids = np.concatenate([np.full(n, e, dtype=np.int32) for e, n in enumerate(rows_per_expert)])
+    ids = np.random.default_rng(seed).permutation(ids)[:, None].astype(np.int32)
+    perm = O.permute(ids, E, None)
+    return dt, x, w1, w3, w2, perm
+
+
+@pytest.mark.parametrize("dtype,act,gather", [
+    ("bf16", "swiglu", False), ("bf16", "gelu", False), ("bf16", "swiglu", True),
+    ("bf16", "gelu", True), ("f32", "swiglu", True), ("f32", "gelu", False),
+])
+@pytest.mark.parametrize("shape", [
+    (4, [0, 1, 130, 257], 256, 384),       # empty expert, 1-row expert, ragged m tiles
+    (3, [200, 64, 129], 200, 136),         # K tail (200 % 64), N tail (136 % 128)
+    (2, [300, 45], 512, 1376),             # F of the 32-expert workload (N tail 1376 % 256)
+])
+def test_grouped_ffn(dtype, act, gather, shape):
+    E, rows, H, F = shape
+    dt, x, w1, w3, w2, perm = _ffn_case(dtype, act, E, rows, H, F)
+    xo = as_np(x)
+    ref = O.grouped_ffn(xo, perm, as_np(w1), None if w3 is None else as_np(w3), as_np(w2), act,
+                        dtype, E)
+    offs = torch.from_numpy(perm["offsets"].astype(np.int32)).cuda()
+    rt = torch.from_numpy(perm["row_token"].astype(np.int32)).cuda()
+    if gather:
+        y = B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
+                            x=x.cuda(), row_token=rt)
+    else:
+        x_perm = x[torch.from_numpy(perm["row_token"])].contiguous().cuda()
+        y = B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
+                            x_perm=x_perm)
+    torch.cuda.synchronize()
+    assert rel_err(as_np(y)[:perm["R"]], ref) <= TOL[dtype]
+
+
+def test_grouped_ffn_identity_and_gemm_only_rows():
+    dt, x, *_ , perm = _ffn_case("bf16", "gelu", 3, [5, 0, 70], 64, 64)
+    offs = torch.from_numpy(perm["offsets"].astype(np.int32)).cuda()
+    rt = torch.from_numpy(perm["row_token"].astype(np.int32)).cuda()
+    y = B().grouped_ffn(offs, None, None, None, "identity", x=x.cuda(), row_token=rt)
+    np.testing.assert_array_equal(as_np(y), as_np(x)[perm["row_token"]])
+
+
+# ---------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("T,H,k", [(1, 8, 1), (1000, 2048, 2), (333, 136, 4), (64, 4096, 8)])
+def test_combine(dtype, T, H, k):
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    R = T * k
+    y = synth.normal(5, 0, (R, H), 1.0, dt)
+    rng = np.random.default_rng(T)
+    row_map = rng.permutation(R).reshape(T, k).astype(np.int32)
+    row_map[rng.random((T, k)) < 0.1] = -1          # some dropped slots
+    gate = torch.from_numpy(rng.random((T, k)).astype(np.float32))
+    out = B().unpermute_combine(y.cuda(), gate.cuda(), torch.from_numpy(row_map).cuda())
+    ref = O.combine(as_np(y), gate.numpy(), row_map, dtype)
+    assert rel_err(as_np(out), ref) <= (1e-6 if dtype == "f32" else 8e-3)
+    # deterministic: a second run is bit-identical
+    out2 = B().unpermute_combine(y.cuda(), gate.cuda(), torch.from_numpy(row_map).cuda())
+    assert torch.equal(out, out2)
