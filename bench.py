@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the grouped GEMM kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source they were taken on; None until captured.
-NCU_TRAFFIC = {"source_sha": None, "bytes_per_forward": None}
+NCU_TRAFFIC = {"source_sha": "ea0e89b397b70f9d", "bytes_per_forward": 897.3e6}
 
 
 def parse_args(argv=None):

@@ -138,7 +138,8 @@ def _ffn_case(dtype, act, E, rows_per_expert, H, F, seed=11):
 @pytest.mark.parametrize("dtype,act,gather", [
     ("bf16", "swiglu", False), ("bf16", "gelu", False), ("bf16", "swiglu", True),
     ("bf16", "gelu", True), ("f32", "swiglu", True), ("f32", "gelu", False),
-])
+], ids=["bf16-swiglu-dense", "bf16-gelu-dense", "bf16-swiglu-gather", "bf16-gelu-gather",
+        "f32-swiglu-gather", "f32-gelu-dense"])
 @pytest.mark.parametrize("shape", [
     (4, [0, 1, 130, 257], 256, 384),       # empty expert, 1-row expert, ragged m tiles
     (3, [200, 64, 129], 200, 136),         # K tail (200 % 64), N tail (136 % 128)
