@@ -101,6 +101,27 @@ moe_status moe_permute(const void* x, const int32_t* token_expert_idx,
                        int32_t* row_token, int32_t* row_map,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute for callers that cannot allocate device memory (no counterpart on
+ * the pages: it exists for hosts such as an engine plugin that must run on
+ * memory planned before the model starts, or a serving process that reserved
+ * its whole device budget up front, where neither cudaMalloc nor a caller
+ * workspace is available).  Same inputs, outputs and results as moe_permute,
+ * but its scratch (status word + per-tile expert histogram) lives in a 1 MiB
+ * array of device memory owned by the library, held by every GPU that loads
+ * the library until exit.  Limit: ceil(T/128) * E <= 262080, else
+ * MOE_ERR_UNSUPPORTED before any launch.  status_out (device int32, nullable)
+ * receives MOE_OK or the first kernel-detected error (MOE_ERR_INDEX_OUT_OF_RANGE);
+ * when NULL such errors are not reported (the pairs are still dropped).  All
+ * calls on a device share the array: calls whose kernels overlap on the GPU
+ * (e.g. two unordered streams) race.  The first call on a device looks up the
+ * array's device address with that device current; make it before any stream
+ * capture.  Allocates nothing (no cudaMalloc/cudaFree).                     */
+moe_status moe_permute_noalloc(const void* x, const int32_t* token_expert_idx,
+                               int T, int H, int E, int top_k, float capacity_factor,
+                               moe_dtype dt, void* x_perm, int32_t* expert_counts,
+                               int32_t* expert_offsets, int32_t* row_token, int32_t* row_map,
+                               int32_t* status_out, moe_stream_t stream);
+
 /* Grouped expert FFN.  [P4] §3 (x times expert_weight[num_experts, hidden,
  * intermediate], then activation and down-projection), §4 (npu_moe_matmul);
  * [P1] §2.2 (one batched GEMM instead of one launch per expert).

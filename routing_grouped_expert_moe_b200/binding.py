@@ -38,6 +38,7 @@ _SIGS = {
     "moe_route": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     "moe_route_from_logits": (_i, [_p, _i, _i, _i, _p, _p, _p]),
     "moe_permute": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_permute_noalloc": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_grouped_ffn": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _sz,
                              _p]),
     "moe_unpermute_combine": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p]),
@@ -173,6 +174,35 @@ def permute(token_expert_idx, num_experts, capacity_factor=0.0, x=None, ws=None)
                             _stream()), "moe_permute")
     out = {"counts": counts, "offsets": offsets, "row_token": row_token, "row_map": row_map,
            "ws": ws}
+    if x_perm is not None:
+        out["x_perm"] = x_perm
+    return out
+
+
+def permute_noalloc(token_expert_idx, num_experts, capacity_factor=0.0, x=None,
+                    status_out=None):
+    """moe_permute without a workspace (library-owned scratch); same outputs as permute()."""
+    _need(token_expert_idx, "token_expert_idx", dtype=torch.int32, dim=2)
+    T, k = token_expert_idx.shape
+    dev = token_expert_idx.device
+    E = int(num_experts)
+    if x is not None:
+        _need(x, "x", dim=2)
+        H, dt = x.shape[1], _dt(x)
+    else:
+        H, dt = 8, BF16
+    if status_out is not None:
+        _need(status_out, "status_out", dtype=torch.int32)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_token = torch.full((T * k,), -1, dtype=torch.int32, device=dev)
+    row_map = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, H, dtype=x.dtype, device=dev) if x is not None else None
+    _check(_lib.moe_permute_noalloc(_ptr(x), _ptr(token_expert_idx), T, H, E, k,
+                                    ctypes.c_float(capacity_factor), dt, _ptr(x_perm),
+                                    _ptr(counts), _ptr(offsets), _ptr(row_token), _ptr(row_map),
+                                    _ptr(status_out), _stream()), "moe_permute_noalloc")
+    out = {"counts": counts, "offsets": offsets, "row_token": row_token, "row_map": row_map}
     if x_perm is not None:
         out["x_perm"] = x_perm
     return out
