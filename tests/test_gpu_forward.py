@@ -56,8 +56,10 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("variant", ["1", "2"], ids=["cta1", "cta2"])
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_forward_small_full_compare(cfg):
+def test_forward_small_full_compare(cfg, variant, monkeypatch):
+    monkeypatch.setenv("MOE_GEMM_VARIANT", variant)
     d = gapped_inputs(cfg)
     out, idx, cnt, _ = _run(cfg, d)
     ref = O.moe_forward(as_np(d["x"]), as_np(d["w_gate"]),

@@ -144,8 +144,13 @@ def _ffn_case(dtype, act, E, rows_per_expert, H, F, seed=11):
     (4, [0, 1, 130, 257], 256, 384),       # empty expert, 1-row expert, ragged m tiles
     (3, [200, 64, 129], 200, 136),         # K tail (200 % 64), N tail (136 % 128)
     (2, [300, 45], 512, 1376),             # F of the 32-expert workload (N tail 1376 % 256)
+    (5, [512, 640, 383, 0, 129], 384, 512),   # even / odd m-tile counts per expert
 ])
-def test_grouped_ffn(dtype, act, gather, shape):
+@pytest.mark.parametrize("variant", ["1", "2"], ids=["cta1", "cta2"])
+def test_grouped_ffn(dtype, act, gather, shape, variant, monkeypatch):
+    if dtype == "f32" and variant == "2":
+        pytest.skip("the fp32 path has a single CUDA-core kernel")
+    monkeypatch.setenv("MOE_GEMM_VARIANT", variant)
     E, rows, H, F = shape
     dt, x, w1, w3, w2, perm = _ffn_case(dtype, act, E, rows, H, F)
     xo = as_np(x)
