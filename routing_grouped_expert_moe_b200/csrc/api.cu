@@ -35,11 +35,11 @@ int num_sms_current() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace: [status | topk_idx | topk_gate | tile_counts | counts | offsets |
-//             row_token | row_map | x_perm | h | y | x_stage | out_stage]
+// Workspace: [status | topk_idx | topk_gate | tile_counts | tickets | partials |
+//             counts | offsets | row_token | row_map | x_perm | h | y | x_stage | out_stage]
 struct WsLayout {
-  size_t status, topk_idx, topk_gate, tile_counts, counts, offsets, row_token, row_map, x_perm,
-      h, y, x_stage, out_stage, total;
+  size_t status, topk_idx, topk_gate, tile_counts, tickets, partials, counts, offsets, row_token,
+      row_map, x_perm, h, y, x_stage, out_stage, total;
 };
 
 WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt, bool host_stage) {
@@ -52,6 +52,8 @@ WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt,
   L.topk_idx = o;    o = align_up(o + R * 4);
   L.topk_gate = o;   o = align_up(o + R * 4);
   L.tile_counts = o; o = align_up(o + tiles * E * 4);
+  L.tickets = o;     o = align_up(o + (static_cast<size_t>(T) / 128 + 1) * 4);
+  L.partials = o;    o = align_up(o + static_cast<size_t>(kRouteMaxCtas) * 128 * E * 4);
   L.counts = o;      o = align_up(o + static_cast<size_t>(E) * 4);
   L.offsets = o;     o = align_up(o + static_cast<size_t>(E + 1) * 4);
   L.row_token = o;   o = align_up(o + R * 4);
@@ -173,7 +175,7 @@ moe_status moe_route(const void* x, const void* w_gate, const float* gate_bias, 
   a.T = T; a.H = H; a.E = E; a.top_k = top_k; a.dt_bf16 = dt == MOE_BF16;
   a.topk_idx = topk_idx; a.topk_gate = topk_gate; a.logits_out = logits_out;
   a.tile_counts = nullptr;
-  const RoutePlan p = route_plan(T, H, E, a.dt_bf16, num_sms_current());
+  const RoutePlan p = route_plan(T, H, E, a.dt_bf16, num_sms_current(), false);
   return cuda_status(launch_route(a, p, as_stream(stream)));
 }
 
@@ -211,6 +213,9 @@ moe_status moe_permute(const void* x, const int32_t* token_expert_idx, int T, in
   p.T = T; p.k = top_k; p.E = E;
   p.BT = kPermuteBT;
   p.tiles = (T + kPermuteBT - 1) / kPermuteBT;
+  p.split = 1;
+  if (x_perm)
+    while (p.split < 16 && p.tiles * p.split < 2 * num_sms_current()) p.split *= 2;
   p.cap = capacity_of(capacity_factor, T, top_k, E);
   p.tile_counts = at<int>(ws, L.tile_counts);
   p.counts = expert_counts; p.offsets = expert_offsets;
@@ -319,7 +324,8 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   void* x_perm = bf16 ? at<void>(ws, L.x_perm) : nullptr;
 
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], s) : cudaSuccess; };
-  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  int* tickets = at<int>(ws, L.tickets);
+  if (launch_clear_status(status, s, tickets, T / 128 + 1) != cudaSuccess) return MOE_ERR_CUDA;
   // 1. route (+ per-tile histogram)
   if (mark(0) != cudaSuccess) return MOE_ERR_CUDA;
   RouteArgs ra{};
@@ -327,7 +333,10 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   ra.T = T; ra.H = H; ra.E = E; ra.top_k = top_k; ra.dt_bf16 = bf16;
   ra.topk_idx = topk_idx; ra.topk_gate = topk_gate; ra.logits_out = nullptr;
   ra.tile_counts = at<int>(ws, L.tile_counts);
-  const RoutePlan rp = route_plan(T, H, E, bf16, nsm);
+  ra.status = status;
+  ra.partials = at<float>(ws, L.partials);
+  ra.tickets = tickets;
+  const RoutePlan rp = route_plan(T, H, E, bf16, nsm, true);
   if (launch_route(ra, rp, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (mark(1) != cudaSuccess) return MOE_ERR_CUDA;
   // 2. scan + scatter over the router's token tiles
@@ -335,6 +344,10 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   pa.idx = topk_idx;
   pa.T = T; pa.k = top_k; pa.E = E;
   pa.BT = rp.BT; pa.tiles = rp.tiles;
+  // enough scatter CTAs to keep the x_perm row copies near HBM bandwidth
+  pa.split = 1;
+  if (x_perm)
+    while (pa.split < 16 && pa.tiles * pa.split < 2 * nsm) pa.split *= 2;
   pa.cap = capacity_of(capacity_factor, T, top_k, E);
   pa.tile_counts = ra.tile_counts;
   pa.counts = counts; pa.offsets = offsets; pa.row_token = row_token; pa.row_map = row_map;

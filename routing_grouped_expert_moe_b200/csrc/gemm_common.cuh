@@ -16,7 +16,7 @@ constexpr int G_A_BYTES = G_BM * G_BK * 2;       // 16 KB
 constexpr int G_BCHUNK = 64 * G_BK * 2;          // one 64-column box: 8 KB
 constexpr int G_B_BYTES = G_ACC_N * G_BK * 2;    // 32 KB
 constexpr int G_STAGE_BYTES = G_A_BYTES + G_B_BYTES;
-constexpr int G_THREADS = 192;
+constexpr int G_THREADS = 320;  // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
 constexpr int G_SMEM = G_STAGES * G_STAGE_BYTES + 1024;
 constexpr uint32_t G_TMEM_COLS = 512;
 

@@ -22,8 +22,10 @@
 // Modes: 0 = gelu(A W1), 1 = silu(A W1) * (A W3) with W1 and W3 side by side in
 // one N=256 MMA (128 output columns), 2 = A W (down-projection).
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
-// owner), warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
+// owner), warps 2-9 epilogue (TMEM lane quarter = warp % 4; two warps per
+// quarter split the tile's columns, so the activation epilogue of one tile
+// finishes within the next tile's main loop).
 #include <cstdlib>
 
 #include "gemm_common.cuh"
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 128);
+      mbar_init(&tempty_bar[i], 256);
     }
     abort_s = 0;
     fence_mbar_init();
@@ -195,7 +197,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
       if (MODE == 1) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
           float g[32], u[32];
           tmem_ld32(t_row + c * 32, g);
           tmem_ld32(t_row + 128 + c * 32, u);
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
           float v[32];
           tmem_ld32(t_row + c * 32, v);
           tmem_ld_wait();

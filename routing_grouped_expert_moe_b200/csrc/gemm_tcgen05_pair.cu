@@ -9,10 +9,10 @@
 // 128-row m-tiles of the same expert (an odd last m-tile leaves the second
 // CTA's rows empty: computed, never stored).
 //
-// Roles per CTA (192 threads): warp 0 TMA producer (both CTAs; completion is
+// Roles per CTA (320 threads): warp 0 TMA producer (both CTAs; completion is
 // counted on the first CTA's full barrier), warp 1 MMA issuer (first CTA only)
-// and TMEM owner (both: the pair allocates together), warps 2-5 epilogue of the
-// CTA's own 128 TMEM lanes.  The first CTA's commits arrive on both CTAs'
+// and TMEM owner (both: the pair allocates together), warps 2-9 epilogue of the
+// CTA's own 128 TMEM lanes (two warps per lane quarter, half the columns each).  The first CTA's commits arrive on both CTAs'
 // "stage free" and "accumulator full" barriers; both CTAs' epilogues arrive on
 // the first CTA's "accumulator free" barrier.
 #include "gemm_common.cuh"
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(&tempty_bar[i], 16);  // one arrival per epilogue warp of both CTAs
     }
     abort_s = 0;
     fence_mbar_init();
@@ -216,7 +216,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
+    const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
       if (MODE == 1) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
           float g[32], u[32];
           tmem_ld32(t_row + c * 32, g);
           tmem_ld32(t_row + 128 + c * 32, u);
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
           float v[32];
           tmem_ld32(t_row + c * 32, v);
           tmem_ld_wait();

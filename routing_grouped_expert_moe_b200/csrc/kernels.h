@@ -20,19 +20,23 @@ struct RouteArgs {
   float* topk_gate;     // [T,k]
   float* logits_out;    // [T,E] or null
   int* tile_counts;     // [tiles,E] or null: per-tile expert histogram
+  int* status;          // device status word or null (pipeline-wait timeouts)
+  float* partials;      // split-H partial logits [tiles, S, 128, E] (tcgen05 path, S > 1)
+  int* tickets;         // [tiles] arrival counters, zero between calls (S > 1)
 };
 
 struct RoutePlan {
-  int kind;   // 0 = SIMT, 1 = tensor-core (mma.sync) path
-  int MT;     // 16-token m-tiles per CTA (tensor-core path)
-  int NTP;    // 8-expert n-tiles, rounded up to a power of two
+  int kind;   // 0 = CUDA cores (fp32, or E not a multiple of 8), 2 = tcgen05
+  int NPAD;   // tcgen05 path: experts padded to the MMA N (64, 128 or 256)
   int BT;     // tokens per CTA tile
   int tiles;  // CTA tiles along T
-  int ck;     // CTAs per cluster splitting H
+  int ck;     // CTAs splitting H per token tile (tcgen05 path)
 };
 
-RoutePlan route_plan(int T, int H, int E, int dt_bf16, int num_sms);
+RoutePlan route_plan(int T, int H, int E, int dt_bf16, int num_sms, bool can_split);
 cudaError_t launch_route(const RouteArgs& a, const RoutePlan& p, cudaStream_t s);
+cudaError_t launch_route_tc(const RouteArgs& a, const RoutePlan& p, cudaStream_t s);
+constexpr int kRouteMaxCtas = 600;  // cap on tiles * split (sizes the partial-logit buffer)
 cudaError_t launch_route_from_logits(const RouteArgs& a, const float* logits, cudaStream_t s);
 
 // ---------------------------------------------------------------- permute
@@ -41,6 +45,7 @@ struct PermuteArgs {
   int T, k, E;
   int BT;               // tokens per tile (must match the histogram's tiling)
   int tiles;
+  int split;            // CTAs per tile in the scatter (share the x_perm row copies)
   int cap;              // per-expert capacity (INT32_MAX when unlimited)
   int* tile_counts;     // [tiles,E] histogram in, tile bases out (in place)
   int32_t* counts;      // [E]   pre-drop counts
@@ -93,6 +98,7 @@ cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_
                            int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- misc
-cudaError_t launch_clear_status(int* status, cudaStream_t s);
+// Clears the status word and n counters (the router's tickets).
+cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters = nullptr, int n = 0);
 
 }  // namespace moe

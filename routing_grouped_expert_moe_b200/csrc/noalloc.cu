@@ -106,6 +106,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, const int32_t* token_ex
   p.E = E;
   p.BT = kPermuteBT;
   p.tiles = tiles;
+  p.split = 1;
   if (capacity_factor > 0.f) {  // C = ceil(cf * T * k / E), at least 1
     const double c =
         std::ceil(static_cast<double>(capacity_factor) * static_cast<double>(T) * top_k / E);

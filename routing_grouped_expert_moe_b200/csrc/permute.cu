@@ -51,42 +51,50 @@ __global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
 
 // One CTA: per-expert exclusive scan over tiles (written back in place as
 // tile bases), pre-drop counts, kept = min(count, C), offsets = scan(kept).
+// Thread (p, e) owns a contiguous run of tiles of expert e: it sums the run,
+// one block scan over p gives each run's base, and a second pass writes the
+// bases; consecutive threads read consecutive experts of a tile (coalesced).
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) k_scan(PermuteArgs a) {
   __shared__ int buf[kScanThreads];
-  __shared__ int carry[kMaxE];
+  __shared__ int total[kMaxE];
   int Ep = 1;
   while (Ep < a.E) Ep <<= 1;
-  const int P = kScanThreads / Ep;  // tiles handled per round
+  const int P = kScanThreads / Ep;  // runs per expert
   const int e = threadIdx.x % Ep, p = threadIdx.x / Ep;
-  for (int i = threadIdx.x; i < a.E; i += kScanThreads) carry[i] = 0;
+  const int run = (a.tiles + P - 1) / P;
+  const int j0 = p * run, j1 = min(a.tiles, j0 + run);
+  int sum = 0;
+  if (e < a.E)
+    for (int j = j0; j < j1; ++j) sum += a.tile_counts[static_cast<size_t>(j) * a.E + e];
+  buf[threadIdx.x] = sum;
   __syncthreads();
-  for (int base = 0; base < a.tiles; base += P) {
-    const int j = base + p;
-    const bool ok = (e < a.E) && (j < a.tiles);
-    const int v = ok ? a.tile_counts[static_cast<size_t>(j) * a.E + e] : 0;
-    buf[threadIdx.x] = v;
+  for (int off = 1; off < P; off <<= 1) {
+    const int u = (p >= off) ? buf[threadIdx.x - off * Ep] : 0;
     __syncthreads();
-    for (int off = 1; off < P; off <<= 1) {
-      const int u = (p >= off) ? buf[threadIdx.x - off * Ep] : 0;
-      __syncthreads();
-      buf[threadIdx.x] += u;
-      __syncthreads();
-    }
-    if (ok) a.tile_counts[static_cast<size_t>(j) * a.E + e] = carry[e] + buf[threadIdx.x] - v;
-    __syncthreads();
-    if (p == P - 1 && e < a.E) carry[e] += buf[threadIdx.x];
+    buf[threadIdx.x] += u;
     __syncthreads();
   }
+  if (e < a.E) {
+    int base = buf[threadIdx.x] - sum;  // exclusive prefix of this run
+    for (int j = j0; j < j1; ++j) {
+      const size_t i = static_cast<size_t>(j) * a.E + e;
+      const int v = a.tile_counts[i];
+      a.tile_counts[i] = base;
+      base += v;
+    }
+    if (p == P - 1) total[e] = buf[threadIdx.x];
+  }
+  __syncthreads();
   if (threadIdx.x < 32) {
-    int run = 0;
+    int acc = 0;
     for (int b = 0; b < a.E; b += 32) {
       const int ee = b + threadIdx.x;
       int kept = 0;
       if (ee < a.E) {
-        a.counts[ee] = carry[ee];
-        kept = min(carry[ee], a.cap);
+        a.counts[ee] = total[ee];
+        kept = min(total[ee], a.cap);
       }
       int incl = kept;
 #pragma unroll
@@ -94,10 +102,10 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(PermuteArgs a) {
         const int u = __shfl_up_sync(0xffffffffu, incl, off);
         if (threadIdx.x >= off) incl += u;
       }
-      if (ee < a.E) a.offsets[ee] = run + incl - kept;
-      run += __shfl_sync(0xffffffffu, incl, 31);
+      if (ee < a.E) a.offsets[ee] = acc + incl - kept;
+      acc += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (threadIdx.x == 0) a.offsets[a.E] = run;
+    if (threadIdx.x == 0) a.offsets[a.E] = acc;
   }
 }
 
@@ -111,7 +119,8 @@ __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
   __shared__ int running[kMaxE];
   __shared__ int rows_s[kScatterMaxPairs];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x;
+  const int split = a.split > 0 ? a.split : 1;
+  const int j = blockIdx.x / split, part = blockIdx.x % split;  // tile, share of its copies
   const int a0 = j * a.BT * a.k;
   const int a1 = min(a.T, (j + 1) * a.BT) * a.k;
   for (int i = threadIdx.x; i < a.E; i += kPermThreads) running[i] = 0;
@@ -147,19 +156,22 @@ __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
         const int rank = a.tile_counts[static_cast<size_t>(j) * a.E + e] + wcnt[warp][e] + rank_w;
         if (rank < a.cap) {
           row = a.offsets[e] + rank;
-          a.row_token[row] = i / a.k;
+          if (part == 0) a.row_token[row] = i / a.k;
         }
       }
-      a.row_map[i] = row;
+      if (part == 0) a.row_map[i] = row;
       rows_s[i - a0] = row;
     }
     __syncthreads();
   }
   if (a.x_perm == nullptr) return;
-  // Gather the kept rows of x into x_perm: one warp per pair, 16-byte vectors.
+  // Gather the kept rows of x into x_perm: this CTA's share of the tile's
+  // pairs, one warp per pair, 16-byte vectors.
   const int row_bytes = a.H * a.elem_bytes;
   const int vecs = row_bytes / 16;
-  for (int p = a0 + warp; p < a1; p += kPermThreads / 32) {
+  const int share = (a1 - a0 + split - 1) / split;
+  const int p0 = a0 + part * share, p1 = min(a1, p0 + share);
+  for (int p = p0 + warp; p < p1; p += kPermThreads / 32) {
     const int row = rows_s[p - a0];
     if (row < 0) continue;
     const int t = p / a.k;
@@ -183,14 +195,18 @@ cudaError_t launch_scan(const PermuteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s) {
   if (a.BT * a.k > kScatterMaxPairs) return cudaErrorInvalidValue;
-  k_scatter<<<a.tiles, kPermThreads, 0, s>>>(a);
+  k_scatter<<<a.tiles * (a.split > 0 ? a.split : 1), kPermThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
-__global__ void k_clear_status(int* status) { *status = 0; }
+__global__ void k_clear_status(int* status, int* counters, int n) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    counters[i] = 0;
+}
 
-cudaError_t launch_clear_status(int* status, cudaStream_t s) {
-  k_clear_status<<<1, 1, 0, s>>>(status);
+cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters, int n) {
+  k_clear_status<<<1, 256, 0, s>>>(status, counters, counters ? n : 0);
   return cudaGetLastError();
 }
 

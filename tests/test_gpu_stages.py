@@ -41,7 +41,10 @@ def test_route_from_logits_bit_exact(T, E, k):
 @pytest.mark.parametrize("dtype,T,H,E,k", [
     ("bf16", 1000, 512, 8, 2), ("bf16", 333, 1024, 32, 2), ("bf16", 517, 256, 128, 2),
     ("bf16", 64, 4096, 8, 2),                       # few tiles: H split over a cluster
-    ("bf16", 96, 200, 16, 4),                       # H not a multiple of the 128 chunk
+    ("bf16", 96, 200, 16, 4),                       # H not a multiple of the 64-wide k-block
+    ("bf16", 20000, 128, 8, 2),                     # enough tiles: no H split
+    ("bf16", 300, 256, 256, 8),                     # 256 experts (MMA N = 256), top-8
+    ("bf16", 19000, 192, 128, 2),                   # 128 experts, no H split, ragged tail
     ("bf16", 50, 64, 12, 3),                        # E not a multiple of 8 (CUDA-core path)
     ("f32", 257, 128, 4, 2), ("f32", 100, 96, 40, 3),
 ])
