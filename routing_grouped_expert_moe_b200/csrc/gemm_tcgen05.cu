@@ -35,7 +35,8 @@ namespace moe {
 template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(G_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
-              const __grid_constant__ CUtensorMap tmB3, const GemmArgs args) {
+              const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmO,
+              const GemmArgs args) {
   constexpr int BN_OUT = ModeCfg<MODE>::BN_OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
+    uint8_t* stg = smem + G_STAGES * G_STAGE_BYTES + (warp - 2) * G_STG_BYTES;  // this warp's staging box
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * G_ACC_N);
       const bool row_ok = row < ti.rows;
+      const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
       if (MODE == 1) {
@@ -221,8 +224,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           tmem_ld32(t_row + c * 32, g);
           tmem_ld32(t_row + 128 + c * 32, u);
           tmem_ld_wait();
-          const int cols_left = args.N - (ti.n0 + c * 32);
-          if (row_ok && cols_left > 0) epilogue_store<1>(g, u, orow + c * 32, cols_left);
+          epilogue_chunk<1>(g, u, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32, args.N,
+                            row_ok ? orow + c * 32 : nullptr, row_ok);
         }
       } else {
 #pragma unroll 1
@@ -230,14 +233,16 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           float v[32];
           tmem_ld32(t_row + c * 32, v);
           tmem_ld_wait();
-          const int cols_left = args.N - (ti.n0 + c * 32);
-          if (row_ok && cols_left > 0) epilogue_store<MODE>(v, v, orow + c * 32, cols_left);
+          epilogue_chunk<MODE>(v, v, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32,
+                               args.N, row_ok ? orow + c * 32 : nullptr, row_ok);
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait0();  // this warp's bulk stores are complete
+    __syncwarp();
   }
   __syncthreads();
   if (warp == 1) {
@@ -251,15 +256,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 // ----------------------------------------------------------------------------
 template <int MODE, bool GATHER>
 static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const CUtensorMap& b3,
-                             const GemmArgs& g, int num_sms, cudaStream_t s) {
+                             const CUtensorMap& o, const GemmArgs& g, int num_sms, cudaStream_t s) {
   auto kern = k_gemm_tc<MODE, GATHER>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
-    if (err != cudaSuccess) return err;
-    attr_set = true;
-  }
-  kern<<<num_sms, G_THREADS, G_SMEM, s>>>(a, b1, b3, g);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
+  if (err != cudaSuccess) return err;
+  kern<<<num_sms, G_THREADS, G_SMEM, s>>>(a, b1, b3, o, g);
   return cudaGetLastError();
 }
 
@@ -275,7 +276,7 @@ static int forced_variant() {
 
 cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
                            const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s) {
-  CUtensorMap ma, mb1, mb3;
+  CUtensorMap ma, mb1, mb3, mo;
   // A: [a_rows, K]; dense source uses 128-row boxes, the gathered source 1-row boxes.
   if (!make_map_2d(&ma, a_src, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(g.K),
                    gather ? 1u : static_cast<uint32_t>(G_BM)))
@@ -286,16 +287,18 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
   } else {
     mb3 = mb1;
   }
+  if (!make_map_out(&mo, g.out, static_cast<uint64_t>(g.R_max), static_cast<uint64_t>(g.N)))
+    return cudaErrorInvalidValue;
   int variant = forced_variant();
   if (variant == 0) variant = (g.R_max >= 512 * g.E) ? 2 : 1;
-  if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, g, num_sms, s);
+  if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, mo, g, num_sms, s);
   switch (mode * 2 + (gather ? 1 : 0)) {
-    case 0: return launch_tc<0, false>(ma, mb1, mb3, g, num_sms, s);
-    case 1: return launch_tc<0, true>(ma, mb1, mb3, g, num_sms, s);
-    case 2: return launch_tc<1, false>(ma, mb1, mb3, g, num_sms, s);
-    case 3: return launch_tc<1, true>(ma, mb1, mb3, g, num_sms, s);
-    case 4: return launch_tc<2, false>(ma, mb1, mb3, g, num_sms, s);
-    case 5: return launch_tc<2, true>(ma, mb1, mb3, g, num_sms, s);
+    case 0: return launch_tc<0, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 1: return launch_tc<0, true>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 2: return launch_tc<1, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 3: return launch_tc<1, true>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 4: return launch_tc<2, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 5: return launch_tc<2, true>(ma, mb1, mb3, mo, g, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

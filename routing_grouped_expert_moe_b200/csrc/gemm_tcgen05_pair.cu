@@ -23,7 +23,7 @@ constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = G_BM * G_BK * 2;            // 16 KB: this CTA's 128 rows
 constexpr int P_B_BYTES = (G_ACC_N / 2) * G_BK * 2;   // 16 KB: half of the 256 columns
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;  // 32 KB
-constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + 1024;
+constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + G_EPI_WARPS * G_STG_BYTES + 1024;
 
 struct PairTile {
   int e, n0, m0, rows, seg_start;
@@ -55,7 +55,8 @@ __device__ __forceinline__ PairTile decode_pair(int tau, const int* prefix, cons
 template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(G_THREADS, 1)
     k_gemm_tc_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
-                   const __grid_constant__ CUtensorMap tmB3, const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmO,
+              const GemmArgs args) {
   constexpr int BN_OUT = ModeCfg<MODE>::BN_OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -219,6 +220,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
+    uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES + (warp - 2) * G_STG_BYTES;  // this warp's staging box
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * G_ACC_N);
       const bool row_ok = row < ti.rows;
+      const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
       if (MODE == 1) {
@@ -241,8 +244,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           tmem_ld32(t_row + c * 32, g);
           tmem_ld32(t_row + 128 + c * 32, u);
           tmem_ld_wait();
-          const int cols_left = args.N - (ti.n0 + c * 32);
-          if (row_ok && cols_left > 0) epilogue_store<1>(g, u, orow + c * 32, cols_left);
+          epilogue_chunk<1>(g, u, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32, args.N,
+                            row_ok ? orow + c * 32 : nullptr, row_ok);
         }
       } else {
 #pragma unroll 1
@@ -250,8 +253,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           float v[32];
           tmem_ld32(t_row + c * 32, v);
           tmem_ld_wait();
-          const int cols_left = args.N - (ti.n0 + c * 32);
-          if (row_ok && cols_left > 0) epilogue_store<MODE>(v, v, orow + c * 32, cols_left);
+          epilogue_chunk<MODE>(v, v, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32,
+                               args.N, row_ok ? orow + c * 32 : nullptr, row_ok);
         }
       }
       tc_fence_before();
@@ -259,6 +262,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty_bar[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait0();  // this warp's bulk stores are complete
+    __syncwarp();
   }
   tc_fence_before();
   cluster_sync_all();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
@@ -270,7 +275,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 template <int MODE, bool GATHER>
 static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b1, const CUtensorMap& b3,
-                               const GemmArgs& g, int num_sms, cudaStream_t s) {
+                               const CUtensorMap& o, const GemmArgs& g, int num_sms,
+                               cudaStream_t s) {
   auto kern = k_gemm_tc_pair<MODE, GATHER>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (err != cudaSuccess) return err;
@@ -286,19 +292,20 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b1, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, b1, b3, g);
+  return cudaLaunchKernelEx(&cfg, kern, a, b1, b3, o, g);
 }
 
 cudaError_t launch_gemm_tc_pair(int mode, bool gather, const CUtensorMap& ma,
-                                const CUtensorMap& mb1, const CUtensorMap& mb3, const GemmArgs& g,
-                                int num_sms, cudaStream_t s) {
+                                const CUtensorMap& mb1, const CUtensorMap& mb3,
+                                const CUtensorMap& mo, const GemmArgs& g, int num_sms,
+                                cudaStream_t s) {
   switch (mode * 2 + (gather ? 1 : 0)) {
-    case 0: return launch_pair<0, false>(ma, mb1, mb3, g, num_sms, s);
-    case 1: return launch_pair<0, true>(ma, mb1, mb3, g, num_sms, s);
-    case 2: return launch_pair<1, false>(ma, mb1, mb3, g, num_sms, s);
-    case 3: return launch_pair<1, true>(ma, mb1, mb3, g, num_sms, s);
-    case 4: return launch_pair<2, false>(ma, mb1, mb3, g, num_sms, s);
-    case 5: return launch_pair<2, true>(ma, mb1, mb3, g, num_sms, s);
+    case 0: return launch_pair<0, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 1: return launch_pair<0, true>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 2: return launch_pair<1, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 3: return launch_pair<1, true>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 4: return launch_pair<2, false>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 5: return launch_pair<2, true>(ma, mb1, mb3, mo, g, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

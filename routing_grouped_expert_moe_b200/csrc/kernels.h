@@ -84,8 +84,9 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
                            const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s);
 // CTA-pair variant (cta_group::2), tensor maps prepared by launch_gemm_tc.
 cudaError_t launch_gemm_tc_pair(int mode, bool gather, const CUtensorMap& ma,
-                                const CUtensorMap& mb1, const CUtensorMap& mb3, const GemmArgs& g,
-                                int num_sms, cudaStream_t s);
+                                const CUtensorMap& mb1, const CUtensorMap& mb3,
+                                const CUtensorMap& mo, const GemmArgs& g, int num_sms,
+                                cudaStream_t s);
 // fp32 CUDA-core path (no TF32).
 cudaError_t launch_gemm_simt(int mode, const void* a_src, const void* b1, const void* b3,
                              const GemmArgs& g, int num_sms, cudaStream_t s);
