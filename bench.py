@@ -44,7 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the grouped GEMM kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source they were taken on; None until captured.
-NCU_TRAFFIC = {"source_sha": "ea0e89b397b70f9d", "bytes_per_forward": 897.3e6}
+NCU_TRAFFIC = {"source_sha": "dc42066570eaa02c", "workload": "page1_gelu",
+               "bytes_per_forward": 903.4e6}
 
 
 def parse_args(argv=None):
@@ -84,7 +85,7 @@ def load_peaks():
 
 def gemm_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("gemm_tcgen05.cu", "common.cuh"):
+    for f in ("gemm_tcgen05.cu", "gemm_tcgen05_pair.cu", "gemm_common.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "routing_grouped_expert_moe_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -384,7 +385,7 @@ def main(argv=None):
     rp_gbs = rp_bytes / (rp_ms / 1e3) / 1e9
     comb_gbs = work["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
     traffic = None
-    if NCU_TRAFFIC["source_sha"] == gemm_source_sha():
+    if NCU_TRAFFIC["source_sha"] == gemm_source_sha() and NCU_TRAFFIC["workload"] == cfg.name:
         traffic = NCU_TRAFFIC["bytes_per_forward"]
 
     line = {
@@ -400,7 +401,7 @@ def main(argv=None):
                 "d2h_bytes_per_step": io_bytes, "ms_per_step": float(e2e_t.item()),
                 "entry_point": "moe_forward_host"},
         "gpu_launches": gpu_launches,
-        "roofline": {"kernel": "k_gemm_tc (expert GEMM-1 + GEMM-2)", "bound": "tensor",
+        "roofline": {"kernel": "k_gemm_tc / k_gemm_tc_pair (expert GEMM-1 + GEMM-2)", "bound": "tensor",
                      "achieved": gemm_tflops, "peak": tc, "unit": "TFLOP/s",
                      "frac": gemm_tflops / tc, "peak_source": f"{peak_src} burst bf16",
                      "frac_of_sustained": gemm_tflops / tc_sus,
