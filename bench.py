@@ -259,6 +259,31 @@ def run_reference(args, cfg):
     return 0
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_inputs(cfg: synth.MoEConfig, rank: int) -> dict:
+    """Inputs of one rank: the weights are the same on every rank (same seed, as a
+    replicated layer has), the tokens are the rank's own (a seed offset per rank)."""
+    d = synth.make_inputs(cfg)
+    if rank > 0:
+        d["x"] = synth.normal(cfg.seed + 7919 * rank, synth.STREAM_X, (cfg.T, cfg.H), cfg.x_std,
+                              cfg.torch_dtype)
+    return d
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (the job is as slow as its slowest rank)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms / 1000.0)
+
+
 # ----------------------------------------------------------------------------- main arm
 
 def main(argv=None):
@@ -282,11 +307,7 @@ def main(argv=None):
 
     from routing_grouped_expert_moe_b200 import binding as B
 
-    # inputs: weights shared across ranks (same seed), tokens differ per rank
-    d = synth.make_inputs(cfg)
-    if rank > 0:
-        d["x"] = synth.normal(cfg.seed + 7919 * rank, synth.STREAM_X, (cfg.T, cfg.H), cfg.x_std,
-                              cfg.torch_dtype)
+    d = rank_inputs(cfg, rank)
     g = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
     T, H, F, E, k = cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k
     ws = B.alloc_workspace(B.workspace_bytes(T, H, F, E, k, cfg.act, cfg.torch_dtype), dev)
@@ -330,12 +351,9 @@ def main(argv=None):
         dist.barrier()
     clocks = sampler.stop(t_wall0, t_wall1)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
-    value = T * world * args.steps / (total_ms / 1000.0)
+    value = job_tokens_per_s(T, world, args.steps, total_ms)
     gpu_launches = 7 * args.steps
 
     # ---- per-stage times of the same fused path (events at stage boundaries)
@@ -368,10 +386,8 @@ def main(argv=None):
         torch.cuda.synchronize()
         if i >= 2:
             e2e_ms.append(s0.elapsed_time(s1))
-    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = T * world / (float(e2e_t.item()) / 1000.0)
+    e2e_step_ms = max_over_ranks(statistics.mean(e2e_ms), dist, dev)
+    e2e_value = job_tokens_per_s(T, world, 1, e2e_step_ms)
     io_bytes = T * H * cfg.elem_bytes
 
     peaks, peak_src = load_peaks()
@@ -398,7 +414,7 @@ def main(argv=None):
                    "parallelism": f"replicas x{world} (token data-parallel, no collective)"},
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
-                "d2h_bytes_per_step": io_bytes, "ms_per_step": float(e2e_t.item()),
+                "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_step_ms,
                 "entry_point": "moe_forward_host"},
         "gpu_launches": gpu_launches,
         "roofline": {"kernel": "k_gemm_tc / k_gemm_tc_pair (expert GEMM-1 + GEMM-2)", "bound": "tensor",
