@@ -21,6 +21,8 @@ constexpr int G_EPI_WARPS = 8;
 constexpr int G_STG_BYTES = 32 * 32 * 2;  // one epilogue warp's staging box: 32 rows x 32 bf16
 constexpr int G_SMEM = G_STAGES * G_STAGE_BYTES + G_EPI_WARPS * G_STG_BYTES + 1024;
 constexpr uint32_t G_TMEM_COLS = 512;
+// Default L2 prefetch distance of the GEMM producers, in k-blocks (0: off).
+constexpr int kGemmPrefetchDist = 0;
 
 template <int MODE>
 struct ModeCfg {

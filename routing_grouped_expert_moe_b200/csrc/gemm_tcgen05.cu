@@ -129,11 +129,34 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           r4[j] = i < ti.rows ? args.row_token[ti.m0 + i] : first;
         }
       }
+      // L2 prefetch runs pf_dist k-blocks ahead of the ring, into the CTA's
+      // next tile once this one is covered.
+      const bool has_next = tau + static_cast<int>(gridDim.x) < total;
+      const TileInfo nx = has_next ? decode_tile(tau + gridDim.x, s_prefix, s_seg_start, s_seg_rows,
+                                                 s_mtiles, E, BN_OUT)
+                                   : ti;
+      auto prefetch_kb = [&](const TileInfo& t, int k0) {
+        if (!GATHER) tma_prefetch_l2_2d(&tmA, k0, t.m0);
+        if (MODE == 1) {
+          tma_prefetch_l2_3d(&tmB1, t.n0, k0, t.e);
+          tma_prefetch_l2_3d(&tmB1, t.n0 + 64, k0, t.e);
+          tma_prefetch_l2_3d(&tmB3, t.n0, k0, t.e);
+          tma_prefetch_l2_3d(&tmB3, t.n0 + 64, k0, t.e);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tma_prefetch_l2_3d(&tmB1, t.n0 + 64 * j, k0, t.e);
+        }
+      };
       bool ok = true;
       for (int kb = 0; kb < num_kb; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, args.status);
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        if (lane == 0 && args.pf_dist > 0) {
+          const int j = kb + args.pf_dist;
+          if (j < num_kb) prefetch_kb(ti, j * G_BK);
+          else if (has_next && j - num_kb < num_kb) prefetch_kb(nx, (j - num_kb) * G_BK);
+        }
         uint8_t* sA = smem + stage * G_STAGE_BYTES;
         uint8_t* sB = sA + G_A_BYTES;
         const int k0 = kb * G_BK;
@@ -289,16 +312,26 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
   }
   if (!make_map_out(&mo, g.out, static_cast<uint64_t>(g.R_max), static_cast<uint64_t>(g.N)))
     return cudaErrorInvalidValue;
+  // MOE_GEMM_PF=<k-blocks> sets the L2 prefetch distance (0 turns it off).
+  GemmArgs ga = g;
+  ga.pf_dist = kGemmPrefetchDist;
+  if (const char* e = getenv("MOE_GEMM_PF")) ga.pf_dist = atoi(e) < 0 ? 0 : atoi(e);
+  // MOE_GEMM_CTAS=<n> caps the persistent grid (a measurement aid: how the
+  // GEMM scales with the number of SMs it runs on).
+  if (const char* e = getenv("MOE_GEMM_CTAS")) {
+    const int n = atoi(e);
+    if (n >= 2 && n < num_sms) num_sms = n;
+  }
   int variant = forced_variant();
   if (variant == 0) variant = (g.R_max >= 512 * g.E) ? 2 : 1;
-  if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, mo, g, num_sms, s);
+  if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, mo, ga, num_sms, s);
   switch (mode * 2 + (gather ? 1 : 0)) {
-    case 0: return launch_tc<0, false>(ma, mb1, mb3, mo, g, num_sms, s);
-    case 1: return launch_tc<0, true>(ma, mb1, mb3, mo, g, num_sms, s);
-    case 2: return launch_tc<1, false>(ma, mb1, mb3, mo, g, num_sms, s);
-    case 3: return launch_tc<1, true>(ma, mb1, mb3, mo, g, num_sms, s);
-    case 4: return launch_tc<2, false>(ma, mb1, mb3, mo, g, num_sms, s);
-    case 5: return launch_tc<2, true>(ma, mb1, mb3, mo, g, num_sms, s);
+    case 0: return launch_tc<0, false>(ma, mb1, mb3, mo, ga, num_sms, s);
+    case 1: return launch_tc<0, true>(ma, mb1, mb3, mo, ga, num_sms, s);
+    case 2: return launch_tc<1, false>(ma, mb1, mb3, mo, ga, num_sms, s);
+    case 3: return launch_tc<1, true>(ma, mb1, mb3, mo, ga, num_sms, s);
+    case 4: return launch_tc<2, false>(ma, mb1, mb3, mo, ga, num_sms, s);
+    case 5: return launch_tc<2, true>(ma, mb1, mb3, mo, ga, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

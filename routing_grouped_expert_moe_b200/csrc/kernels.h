@@ -73,6 +73,7 @@ struct GemmArgs {
   int T;                     // rows of the gathered source
   void* out;                 // [R_max, N]
   int* status;
+  int pf_dist;               // k-blocks ahead of the TMA ring to prefetch into L2 (0: off)
 };
 
 struct GemmTcPlan {
