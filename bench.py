@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hbm-copy-sweep", action="store_true",
+                    help="time plain device copies at the memory stages' sizes and exit")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds for the oracle baseline sample")
     return ap.parse_args(argv)
@@ -286,11 +288,39 @@ def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, total_ms: flo
 
 # ----------------------------------------------------------------------------- main arm
 
+def hbm_copy_sweep() -> int:
+    """What a plain device copy achieves at the sizes the memory-bound stages
+    move (L2 cold before each copy), one JSON line per size."""
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for mb in (4, 8, 16, 33, 67, 134, 268, 1024):
+        n = mb * (1 << 20) // 2
+        a = torch.empty(n, dtype=torch.bfloat16, device=dev)
+        b = torch.empty_like(a)
+        ts = []
+        for i in range(13):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            b.copy_(a)
+            s1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(s0.elapsed_time(s1) * 1000.0)
+        us = statistics.median(ts)
+        print(json.dumps({"copy_mb_read": mb, "us": us, "gbs_read_plus_write": 2 * n * 2 / us / 1e3}),
+              flush=True)
+        del a, b
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     cfg = resolve_config(args.config)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.hbm_copy_sweep:
+        return hbm_copy_sweep()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
