@@ -189,8 +189,9 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- oracle timing
 
 def oracle_sample(cfg: synth.MoEConfig, d: dict, n_tokens: int) -> float:
-    """Seconds the CPU oracle takes for the whole layer on the first n_tokens tokens."""
-    from oracle import moe_oracle as O
+    """Seconds the C++ CPU oracle (plain float64 loops, OpenMP over rows) takes for
+    the whole layer on the first n_tokens tokens."""
+    from oracle import moe_oracle_cpp as O
     f = lambda t: None if t is None else t.float().numpy()  # noqa: E731
     x = f(d["x"][:n_tokens])
     t0 = time.perf_counter()
@@ -205,15 +206,10 @@ def _oracle_inputs(cfg, d):
     d["_w1"], d["_w3"], d["_w2"] = f(d["w1"]), f(d["w3"]), f(d["w2"])
 
 
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+def oracle_threads() -> int:
+    """Threads the C++ oracle's OpenMP loops run on."""
+    from oracle import moe_oracle_cpp as O
+    return O.num_threads()
 
 
 def calibrate_tokens(cfg, d, target_s: float) -> tuple[int, float]:
@@ -228,9 +224,9 @@ def calibrate_tokens(cfg, d, target_s: float) -> tuple[int, float]:
 def cpu_baseline(cfg, d, target_s: float) -> dict:
     _oracle_inputs(cfg, d)
     n, dt = calibrate_tokens(cfg, d, target_s)
-    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"whole layer (float64 numpy oracle) on the first {n} of {cfg.T} tokens "
-                      f"of {cfg.name}, {dt:.1f} s"}
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"whole layer (C++ float64 oracle, plain loops, OpenMP) on the first {n} "
+                      f"of {cfg.T} tokens of {cfg.name}, {dt:.1f} s"}
 
 
 def run_reference(args, cfg):
@@ -252,9 +248,10 @@ def run_reference(args, cfg):
             "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {**workload_desc(cfg), "sample_tokens_per_step": n},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(),
                              "kind": "oracle",
-                             "sample": f"{n} of {cfg.T} tokens per step, whole layer"},
+                             "sample": f"{n} of {cfg.T} tokens per step, whole layer, C++ "
+                                       f"float64 oracle (plain loops, OpenMP)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

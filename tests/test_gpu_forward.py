@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from oracle import moe_oracle as O
+from oracle import moe_oracle_cpp as OC
 from routing_grouped_expert_moe_b200 import synth
 from tests.helpers import TOL, as_np, gapped_inputs, rel_err
 
@@ -56,13 +57,14 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("oracle", ["numpy", "cpp"])
 @pytest.mark.parametrize("variant", ["1", "2"], ids=["cta1", "cta2"])
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_forward_small_full_compare(cfg, variant, monkeypatch):
+def test_forward_small_full_compare(cfg, variant, oracle, monkeypatch):
     monkeypatch.setenv("MOE_GEMM_VARIANT", variant)
     d = gapped_inputs(cfg)
     out, idx, cnt, _ = _run(cfg, d)
-    ref = O.moe_forward(as_np(d["x"]), as_np(d["w_gate"]),
+    ref = (O if oracle == "numpy" else OC).moe_forward(as_np(d["x"]), as_np(d["w_gate"]),
                         None if d["gate_bias"] is None else as_np(d["gate_bias"]),
                         as_np(d["w1"]), None if d["w3"] is None else as_np(d["w3"]),
                         as_np(d["w2"]), cfg.top_k, cfg.capacity_factor, cfg.act, cfg.dtype)

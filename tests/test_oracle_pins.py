@@ -14,10 +14,17 @@ import pytest
 import torch
 from scipy.special import expit, softmax
 
-from oracle import moe_oracle as O
+from oracle import moe_oracle as PY
+from oracle import moe_oracle_cpp as CPP
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 rng = np.random.default_rng(12345)
+
+
+@pytest.fixture(params=["numpy", "cpp"])
+def O(request):
+    """Every pin runs on both oracles: the numpy one and the plain C++ one."""
+    return PY if request.param == "numpy" else CPP
 
 
 def _load(name):
@@ -27,13 +34,13 @@ def _load(name):
 
 # ---------------------------------------------------------------- rounding
 
-def test_bf16_rounding_golden():
+def test_bf16_rounding_golden(O):
     for c in _load("bf16_rounding_cases.json")["cases"]:
         got = float(O.round_to_bf16(np.array([c["value"]]))[0])
         assert got == c["expect"], c
 
 
-def test_bf16_rounding_matches_library_on_fp32_values():
+def test_bf16_rounding_matches_library_on_fp32_values(O):
     # fp32 -> bf16 is a single rounding in torch (round to nearest even), so on
     # values exactly representable in fp32 the oracle's one-step rounding must agree.
     v = np.concatenate([
@@ -45,7 +52,7 @@ def test_bf16_rounding_matches_library_on_fp32_values():
     np.testing.assert_array_equal(got, ref)
 
 
-def test_bf16_rounding_subnormal_and_overflow():
+def test_bf16_rounding_subnormal_and_overflow(O):
     assert O.round_to_bf16(np.array([2.0 ** -133]))[0] == 2.0 ** -133
     assert O.round_to_bf16(np.array([2.0 ** -135]))[0] == 0.0          # below half spacing
     assert math.isinf(O.round_to_bf16(np.array([3.5e38]))[0])
@@ -55,7 +62,7 @@ def test_bf16_rounding_subnormal_and_overflow():
 
 # ---------------------------------------------------------------- logits
 
-def test_router_logits_match_library_matmul():
+def test_router_logits_match_library_matmul(O):
     x = torch.randn(37, 96, dtype=torch.float64).to(torch.bfloat16).to(torch.float64)
     w = torch.randn(96, 5, dtype=torch.float64).to(torch.bfloat16).to(torch.float64)
     b = torch.randn(5, dtype=torch.float64).float().double()
@@ -64,7 +71,7 @@ def test_router_logits_match_library_matmul():
     np.testing.assert_array_equal(got, ref)
 
 
-def test_router_logits_orientation_and_bias_exact():
+def test_router_logits_orientation_and_bias_exact(O):
     # Integer inputs: every partial sum is exact, so the result is known exactly.
     x = np.array([[1, 2, 3]], dtype=np.float64)             # [T=1, H=3]
     w = np.array([[1, 0], [0, 1], [1, 1]], dtype=np.float64)  # [H=3, E=2]
@@ -75,30 +82,30 @@ def test_router_logits_orientation_and_bias_exact():
 # ---------------------------------------------------------------- top-k
 
 @pytest.mark.parametrize("E", [2, 3, 4, 5, 6, 8])
-def test_topk_matches_bruteforce(E):
+def test_topk_matches_bruteforce(O, E):
     for k in range(1, min(3, E) + 1):
         lg = rng.standard_normal((200, E)).astype(np.float32)
         idx = O.topk_select(lg, k)
         for t in range(lg.shape[0]):
-            assert tuple(idx[t]) == O.topk_select_bruteforce(lg[t], k)
+            assert tuple(idx[t]) == PY.topk_select_bruteforce(lg[t], k)
             # independent check: the chosen set has the largest sum over all subsets
             best = max(combinations(range(E), k), key=lambda s: sum(float(lg[t, e]) for e in s))
             assert set(idx[t]) == set(best)
 
 
-def test_topk_k_equals_E_is_descending_sort():
+def test_topk_k_equals_E_is_descending_sort(O):
     lg = rng.standard_normal((50, 7)).astype(np.float32)
     idx = O.topk_select(lg, 7)
     np.testing.assert_array_equal(idx, np.argsort(-lg, axis=1, kind="stable"))
 
 
-def test_topk_k1_is_argmax_with_low_id_ties():
+def test_topk_k1_is_argmax_with_low_id_ties(O):
     lg = rng.integers(0, 3, (300, 6)).astype(np.float32)     # many ties
     idx = O.topk_select(lg, 1)
     np.testing.assert_array_equal(idx[:, 0], np.argmax(lg, axis=1))
 
 
-def test_topk_ties_and_nan():
+def test_topk_ties_and_nan(O):
     lg = np.array([[1.0, 2.0, 2.0, 0.5],
                    [np.nan, -np.inf, 1.0, np.nan]], dtype=np.float32)
     idx = O.topk_select(lg, 4)
@@ -108,7 +115,7 @@ def test_topk_ties_and_nan():
 
 # ---------------------------------------------------------------- gates
 
-def test_gates_sum_to_one_and_closed_forms():
+def test_gates_sum_to_one_and_closed_forms(O):
     lg = (rng.standard_normal((500, 8)) * 3).astype(np.float32)
     for k in (1, 2, 3):
         idx = O.topk_select(lg, k)
@@ -122,7 +129,7 @@ def test_gates_sum_to_one_and_closed_forms():
             np.testing.assert_allclose(g[:, 0], expit(sel[:, 0] - sel[:, 1]), rtol=1e-7)
 
 
-def test_gates_equal_full_softmax_then_renormalise():
+def test_gates_equal_full_softmax_then_renormalise(O):
     lg = (rng.standard_normal((300, 16)) * 2).astype(np.float32)
     idx = O.topk_select(lg, 2)
     p = softmax(lg.astype(np.float64), axis=1)               # library softmax over all E
@@ -134,7 +141,7 @@ def test_gates_equal_full_softmax_then_renormalise():
 
 # ---------------------------------------------------------------- dispatch
 
-def test_capacity_values():
+def test_capacity_values(O):
     assert O.capacity(1.2, 4096, 2, 8) == 1229
     assert O.capacity(1.25, 32768, 2, 32) == 2560
     assert O.capacity(0.5, 512, 2, 8) == 64
@@ -147,7 +154,7 @@ def test_capacity_values():
 
 
 @pytest.mark.parametrize("case", _load("capacity_cases.json")["cases"], ids=lambda c: c["name"])
-def test_permute_golden(case):
+def test_permute_golden(O, case):
     idx = np.array(case["topk_idx"], dtype=np.int32)
     cap = O.capacity(case["capacity_factor"], case["T"], case["k"], case["E"])
     assert cap == case["capacity"]
@@ -157,12 +164,12 @@ def test_permute_golden(case):
     assert p["dropped"] == case["dropped"]
 
 
-def test_counts_match_bincount():
+def test_counts_match_bincount(O):
     idx = rng.integers(0, 13, (1000, 3)).astype(np.int32)
     np.testing.assert_array_equal(O.expert_counts(idx, 13), np.bincount(idx.ravel(), minlength=13))
 
 
-def test_index_out_of_range_is_an_error():
+def test_index_out_of_range_is_an_error(O):
     with pytest.raises(O.IndexOutOfRange):
         O.permute(np.array([[0, 4]], dtype=np.int32), 4, None)
     with pytest.raises(O.IndexOutOfRange):
@@ -174,7 +181,7 @@ def _distinct_ids(T, E, k, skew=0.0):
     return np.stack([rng.choice(E, size=k, replace=False, p=w) for _ in range(T)]).astype(np.int32)
 
 
-def test_permute_no_limit_is_stable_sort_by_expert():
+def test_permute_no_limit_is_stable_sort_by_expert(O):
     T, E, k = 400, 9, 3
     idx = _distinct_ids(T, E, k)
     p = O.permute(idx, E, None)
@@ -185,7 +192,7 @@ def test_permute_no_limit_is_stable_sort_by_expert():
 
 
 @pytest.mark.parametrize("cf", [0.0, 0.5, 0.8, 1.0, 1.3])
-def test_permute_invariants(cf):
+def test_permute_invariants(O, cf):
     T, E, k = 600, 8, 2
     idx = _distinct_ids(T, E, k, skew=0.3)
     cap = O.capacity(cf, T, k, E)
@@ -220,7 +227,7 @@ def test_permute_invariants(cf):
 
 # ---------------------------------------------------------------- expert FFN / combine
 
-def test_activations_match_library():
+def test_activations_match_library(O):
     z = np.linspace(-8, 8, 1001)
     zt = torch.from_numpy(z)
     np.testing.assert_allclose(O.gelu(z), torch.nn.functional.gelu(zt).numpy(), rtol=1e-13, atol=1e-15)
@@ -228,7 +235,7 @@ def test_activations_match_library():
 
 
 @pytest.mark.parametrize("act", ["gelu", "swiglu"])
-def test_single_expert_k1_equals_dense_ffn(act):
+def test_single_expert_k1_equals_dense_ffn(O, act):
     # E=1, k=1, no capacity: every gate is 1 and the layer is the dense FFN.
     T, H, F = 33, 24, 40                                       # H != F: a transpose fails
     x = rng.standard_normal((T, H)).astype(np.float32).astype(np.float64)
@@ -248,7 +255,7 @@ def test_single_expert_k1_equals_dense_ffn(act):
     np.testing.assert_allclose(res["out"], ref, rtol=2e-6, atol=2e-6 * np.abs(ref).max())
 
 
-def test_identity_experts_give_x_times_kept_gate_sum():
+def test_identity_experts_give_x_times_kept_gate_sum(O):
     T, H, E, k = 120, 16, 6, 2
     x = O.round_to_bf16(rng.standard_normal((T, H)))
     lg = rng.standard_normal((T, E)).astype(np.float32)
@@ -265,7 +272,7 @@ def test_identity_experts_give_x_times_kept_gate_sum():
             assert np.all(res["out"][all_dropped] == 0)
 
 
-def test_combine_is_linear_in_y():
+def test_combine_is_linear_in_y(O):
     T, H, k = 50, 8, 2
     row_map = np.arange(T * k).reshape(T, k)
     row_map[3, 1] = -1
@@ -277,7 +284,7 @@ def test_combine_is_linear_in_y():
     np.testing.assert_allclose(lhs, rhs, rtol=1e-5, atol=1e-5)
 
 
-def test_layer_matches_per_token_pseudocode():
+def test_layer_matches_per_token_pseudocode(O):
     """The grouped (permute -> expert loop -> combine) oracle equals the pages'
     per-token form: softmax over all experts, top-k, renormalise, sum of
     gate-weighted expert outputs — written here with torch float64 ops."""
@@ -302,7 +309,7 @@ def test_layer_matches_per_token_pseudocode():
         np.testing.assert_allclose(res["out"][t], acc.numpy(), rtol=1e-5, atol=1e-6)
 
 
-def test_sampled_rows_equal_full_layer():
+def test_sampled_rows_equal_full_layer(O):
     T, H, F, E, k = 64, 16, 32, 4, 2
     x = O.round_to_bf16(rng.standard_normal((T, H)))
     wg = O.round_to_bf16(rng.standard_normal((H, E)) / 4)
@@ -313,3 +320,27 @@ def test_sampled_rows_equal_full_layer():
         toks = np.array([0, 5, 17, 63])
         samp = O.moe_forward_sampled(x, full["logits"], w1, None, w2, k, cf, "gelu", "bf16", toks)
         np.testing.assert_array_equal(samp["out_rows"], full["out"][toks])
+
+
+@pytest.mark.parametrize("act,cf", [("gelu", 0.6), ("swiglu", 0.0)])
+def test_numpy_and_cpp_oracles_agree(act, cf):
+    """The two oracles are written independently (numpy with library matmuls,
+    C++ with plain loops): on the same bf16 inputs they agree exactly on every
+    index, count and gate, and on the outputs up to the rare bf16 rounding
+    decision that a different float64 summation order can flip."""
+    T, H, F, E, k = 96, 64, 80, 8, 2
+    x = PY.round_to_bf16(rng.standard_normal((T, H)))
+    wg = PY.round_to_bf16(rng.standard_normal((H, E)) / 8)
+    w1 = PY.round_to_bf16(rng.standard_normal((E, H, F)) / 8)
+    w3 = PY.round_to_bf16(rng.standard_normal((E, H, F)) / 8) if act == "swiglu" else None
+    w2 = PY.round_to_bf16(rng.standard_normal((E, F, H)) / 9)
+    la, lb = PY.router_logits(x, wg), CPP.router_logits(x, wg)
+    assert np.all(np.abs(la.astype(np.float64) - lb) <= np.spacing(np.abs(la)))
+    a = PY.moe_forward(x, wg, None, w1, w3, w2, k, cf, act, "bf16", logits=la)
+    b = CPP.moe_forward(x, wg, None, w1, w3, w2, k, cf, act, "bf16", logits=la)
+    for key in ("topk_idx", "topk_gate", "counts", "kept", "offsets", "row_token", "row_slot",
+                "row_map"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+    assert a["capacity"] == b["capacity"] and a["dropped"] == b["dropped"]
+    np.testing.assert_allclose(b["out"], a["out"], rtol=2.0 ** -7, atol=1e-30)
+    assert np.mean(a["out"] == b["out"]) > 0.98
