@@ -56,6 +56,10 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["layer", "expert_matmul", "route_stats"], default="layer",
+                    help="layer: the MoE layer (default, the headline); expert_matmul: the k=1\n"
+                         "up-projection op on x[1024,4096] x W[8,4096,14336]; route_stats: the\n"
+                         "router with its load statistics on the e32_long router shape")
     ap.add_argument("--hbm-copy-sweep", action="store_true",
                     help="time plain device copies at the memory stages' sizes and exit")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -311,6 +315,92 @@ def hbm_copy_sweep() -> int:
     return 0
 
 
+def _time_steps(fn, steps: int, warmup: int, flush) -> list:
+    """CUDA-event milliseconds of each of `steps` calls (L2 flushed before each)."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        fn()
+        s1.record()
+        ms.append((s0, s1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ms]
+
+
+def run_op(args) -> int:
+    """One JSON line for a single-op row (not the layer headline)."""
+    from routing_grouped_expert_moe_b200 import binding as B
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_src = load_peaks()
+    steps, warmup = min(args.steps, 100), max(args.warmup, 3)
+    if args.op == "expert_matmul":
+        T, H, I, E, seed = 1024, 4096, 14336, 8, 5001
+        x = synth.normal(seed, synth.STREAM_X, (T, H), 1.0, torch.bfloat16).to(dev)
+        w = synth.normal(seed, synth.STREAM_W1, (E, H, I), H ** -0.5, torch.bfloat16).to(dev)
+        ids = synth.random_expert_ids(seed, T, E, 1)[:, 0].contiguous().to(dev)
+        out = torch.empty(T, I, dtype=torch.bfloat16, device=dev)
+        ws = B.alloc_workspace(B._lib.moe_expert_matmul_workspace_bytes(T, H, I, E, B.BF16), dev)
+        ms = _time_steps(lambda: B.expert_matmul(x, w, ids, out=out, ws=ws), steps, warmup, flush)
+        if B.device_status(ws) != B.OK:
+            raise RuntimeError("expert_matmul device status")
+        t_ms = statistics.mean(ms)
+        flops = 2.0 * T * H * I
+        tflops = flops / (t_ms / 1e3) / 1e12
+        tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        # weights of the experts that received tokens, read once, plus x in and out
+        used = int(torch.unique(ids).numel())
+        nbytes = used * H * I * 2 + T * H * 2 + T * I * 2
+        gbs = nbytes / (t_ms / 1e3) / 1e9
+        # ~T/E rows per expert: below the ridge point the op is bound by the weight stream
+        hbm_bound = flops / nbytes < tc * 1e12 / (hbm * 1e9)
+        line = {"metric": "expert_matmul tokens/s (k=1 up-projection)", "value": T / (t_ms / 1e3),
+                "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+                "ms_per_step": t_ms, "higher_is_better": True, "dtype": "bf16",
+                "data": "synthetic (seeded normal x and weights, uniform expert ids)",
+                "config": {"workload": "expert_matmul_p4", "T": T, "H": H, "I": I, "E": E,
+                           "l2": "flushed before every step"},
+                "roofline": ({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                              "frac": gbs / hbm, "peak_source": peak_src, "algorithmic_bytes": nbytes,
+                              "tflops": tflops, "frac_of_bf16_peak": tflops / tc}
+                             if hbm_bound else
+                             {"bound": "tensor", "achieved": tflops, "peak": tc, "unit": "TFLOP/s",
+                              "frac": tflops / tc, "peak_source": f"{peak_src} burst bf16"}),
+                "note": "whole op (permute + grouped GEMM + unpermute) time"}
+    else:
+        cfg = synth.CONFIGS["e32_long"]
+        d = synth.make_inputs(cfg, with_weights=False)
+        x, wg = d["x"].to(dev), d["w_gate"].to(dev)
+        b = None if d["gate_bias"] is None else d["gate_bias"].to(dev)
+        ws = B.alloc_workspace(B._lib.moe_route_stats_workspace_bytes(cfg.T, cfg.E), dev)
+        ms = _time_steps(lambda: B.route_stats(x, wg, b, cfg.top_k, ws=ws), steps, warmup, flush)
+        if B.device_status(ws) != B.OK:
+            raise RuntimeError("route_stats device status")
+        t_ms = statistics.mean(ms)
+        T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.top_k
+        nbytes = T * H * 2 + H * E * 2 + T * k * 8 + 2 * T * E * 4   # x, W_gate, idx+gate, logits w+r
+        gbs = nbytes / (t_ms / 1e3) / 1e9
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        line = {"metric": "route_stats tokens/s (router + load statistics)", "value": T / (t_ms / 1e3),
+                "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+                "ms_per_step": t_ms, "higher_is_better": True, "dtype": "bf16",
+                "data": "synthetic (seeded Philox normal inputs)",
+                "config": {"workload": "e32_long router", "T": T, "H": H, "E": E, "top_k": k,
+                           "l2": "flushed before every step"},
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                             "frac": gbs / hbm, "peak_source": peak_src, "algorithmic_bytes": nbytes}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     cfg = resolve_config(args.config)
@@ -318,6 +408,8 @@ def main(argv=None):
         return run_reference(args, cfg)
     if args.hbm_copy_sweep:
         return hbm_copy_sweep()
+    if args.op != "layer":
+        return run_op(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

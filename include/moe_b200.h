@@ -184,6 +184,41 @@ moe_status moe_forward_host(const void* x_host, const void* w_gate, const float*
                             moe_act act, moe_dtype dt, void* out_host,
                             void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Router load statistics.  [P3] Step 4 and [P4] §5.3 name an auxiliary
+ * load-balancing loss (--moe-aux-loss-coeff) but not its formula, so the
+ * router's two per-expert statistics are returned instead of a loss:
+ *   expert_counts[e] (int32, pre-drop) = #{(t,s): topk_idx[t,s] = e}
+ *   prob_mean[e]     (fp32)            = (1/T) sum_t softmax_e(logits[t])
+ * with the softmax over all E experts of the fp32 logits moe_route computes
+ * (bias included).  Also writes topk_idx / topk_gate exactly as moe_route.
+ * Both sums run in a fixed order: bit-identical from run to run.  Runs the
+ * router without splitting H across CTAs.  ws: device scratch of at least
+ * moe_route_stats_workspace_bytes(T, E) bytes (256-byte aligned); errors as
+ * moe_route, plus MOE_ERR_WORKSPACE.                                        */
+size_t moe_route_stats_workspace_bytes(int T, int E);
+moe_status moe_route_stats(const void* x, const void* w_gate, const float* gate_bias,
+                           int T, int H, int E, int top_k, moe_dtype dt,
+                           int32_t* topk_idx, float* topk_gate,
+                           int32_t* expert_counts, float* prob_mean,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Per-token expert matmul with one expert per token (top_k = 1, up-projection
+ * only, no activation).  [P4] §3: x[tokens, hidden], expert_weight[num_experts,
+ * hidden, intermediate] and int32 token_expert_idx[tokens] in, [tokens,
+ * intermediate] out; §5.2: ids outside [0, E) are errors, not clamped.
+ *   out[t] = x[t] @ expert_weight[token_expert_idx[t]]   rounded once to dt
+ * out is [T, I] (I = intermediate size, a multiple of 8).  The tokens are
+ * rearranged by expert (the permute step, no capacity limit), multiplied by
+ * the grouped GEMM and put back in token order.  A token whose id is outside
+ * [0, E) gets a zero row in out and the device status becomes
+ * MOE_ERR_INDEX_OUT_OF_RANGE.  ws: device scratch of at least
+ * moe_expert_matmul_workspace_bytes(T, H, I, E, dt) bytes.                   */
+size_t moe_expert_matmul_workspace_bytes(int T, int H, int I, int E, moe_dtype dt);
+moe_status moe_expert_matmul(const void* x, const void* expert_weight,
+                             const int32_t* token_expert_idx, int T, int H, int I, int E,
+                             moe_dtype dt, void* out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the status the kernels of the last
  * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */
 moe_status moe_get_device_status(void* ws, moe_stream_t stream);

@@ -284,6 +284,45 @@ int oracle_combine(const double* y, int H, const float* gates, const int64_t* ro
   return 0;
 }
 
+// prob_mean[e] = (1/T) sum_t softmax(logits[t])[e], the softmax over all E, float64.
+int oracle_router_prob_mean(const float* logits, int T, int E, double* prob_mean) {
+  if (T < 0 || E < 1) return 1;
+  for (int e = 0; e < E; ++e) prob_mean[e] = 0.0;
+  std::vector<double> z(E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + static_cast<int64_t>(t) * E;
+    double mx = -INFINITY;
+    for (int e = 0; e < E; ++e) mx = std::fmax(mx, static_cast<double>(l[e]));
+    double den = 0.0;
+    for (int e = 0; e < E; ++e) { z[e] = std::exp(static_cast<double>(l[e]) - mx); den += z[e]; }
+    for (int e = 0; e < E; ++e) prob_mean[e] += z[e] / den;
+  }
+  if (T > 0)
+    for (int e = 0; e < E; ++e) prob_mean[e] /= T;
+  return 0;
+}
+
+// out[t][i] = sum_j x[t][j] * W[idx[t]][j][i] (float64, j ascending), rounded to dtype.
+// W is [E][H][I]; an id outside [0, E) is an error (status 2).
+int oracle_expert_matmul(const float* x, const float* w, const int32_t* idx, int T, int H, int I,
+                         int E, int dtype, double* out) {
+  for (int t = 0; t < T; ++t)
+    if (idx[t] < 0 || idx[t] >= E) return 2;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < T; ++t) {
+    const float* W = w + static_cast<int64_t>(idx[t]) * H * I;
+    double* o = out + static_cast<int64_t>(t) * I;
+    for (int i = 0; i < I; ++i) o[i] = 0.0;
+    for (int j = 0; j < H; ++j) {
+      const double xj = x[static_cast<int64_t>(t) * H + j];
+      const float* wj = W + static_cast<int64_t>(j) * I;
+      for (int i = 0; i < I; ++i) o[i] += xj * static_cast<double>(wj[i]);
+    }
+    for (int i = 0; i < I; ++i) o[i] = round_to(dtype, o[i]);
+  }
+  return 0;
+}
+
 // Elementwise activation (0: SiLU z / (1 + exp(-z)), 1: exact GELU), float64.
 int oracle_activation(const double* z, int64_t n, int which, double* out) {
   if (which != 0 && which != 1) return 1;

@@ -322,6 +322,47 @@ def combine(y, gates, row_map, dtype: str) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Router load statistics.   [P3] Step 4 / [P4] §5.3 (auxiliary load-balancing
+# loss named, formula not given: the two per-expert statistics it is built from)
+# --------------------------------------------------------------------------
+
+
+def router_load_stats(logits, idx, E: int) -> dict:
+    """counts[e] = pairs routed to e (pre-drop); prob_mean[e] = mean over tokens
+    of softmax(logits[t])[e], the softmax over all E experts, in float64."""
+    lg = np.asarray(logits, dtype=np.float64)
+    T = lg.shape[0]
+    counts = expert_counts(idx, E)
+    prob_sum = np.zeros(E, dtype=np.float64)
+    for t in range(T):
+        z = np.exp(lg[t] - lg[t].max())
+        prob_sum += z / z.sum()
+    return {"counts": counts, "prob_mean": prob_sum / T if T else prob_sum}
+
+
+# --------------------------------------------------------------------------
+# One expert per token, up-projection only.   [P4] §3 (x[tokens, hidden],
+# expert_weight[num_experts, hidden, intermediate], int32 token_expert_idx), §5.2
+# --------------------------------------------------------------------------
+
+
+def expert_matmul(x, expert_weight, token_expert_idx, dtype: str) -> np.ndarray:
+    """out[t] = x[t] @ expert_weight[token_expert_idx[t]], float64 sum, rounded once to dtype."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(expert_weight)
+    ids = np.asarray(token_expert_idx)
+    E = w.shape[0]
+    if ids.size and (ids.min() < 0 or ids.max() >= E):
+        raise IndexOutOfRange("expert id outside [0, E)")
+    out = np.zeros((x.shape[0], w.shape[2]), dtype=np.float64)
+    for e in range(E):
+        rows = np.nonzero(ids == e)[0]
+        if rows.size:
+            out[rows] = x[rows] @ np.asarray(w[e], dtype=np.float64)
+    return round_to(dtype, out)
+
+
+# --------------------------------------------------------------------------
 # The whole layer.   [P3] MoEOperator::Forward; [P5] ch.8 moe_router
 # --------------------------------------------------------------------------
 

@@ -44,6 +44,8 @@ for _name, _args in {
     "oracle_grouped_ffn": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P],
     "oracle_combine": [_P, _I, _P, _P, _I, _I, _I, _P],
     "oracle_activation": [_P, _I64, _I, _P],
+    "oracle_router_prob_mean": [_P, _I, _I, _P],
+    "oracle_expert_matmul": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
     "oracle_num_threads": [],
 }.items():
     _f = getattr(_lib, _name)
@@ -216,6 +218,26 @@ def combine(y, gates, row_map, dtype: str) -> np.ndarray:
     yy, py = _c(y if y.size else np.zeros((1, max(H, 1))), np.float64)
     out = np.zeros((T, H), dtype=np.float64)
     _check(_lib.oracle_combine(py, H, pg, pm, T, k, _DT[dtype], out.ctypes.data_as(_P)), "combine")
+    return out
+
+
+def router_load_stats(logits, idx, E: int) -> dict:
+    lg, pl = _c(logits, np.float32)
+    T = lg.shape[0]
+    prob = np.zeros(E, dtype=np.float64)
+    _check(_lib.oracle_router_prob_mean(pl, T, E, prob.ctypes.data_as(_P)), "router_load_stats")
+    return {"counts": expert_counts(idx, E), "prob_mean": prob}
+
+
+def expert_matmul(x, expert_weight, token_expert_idx, dtype: str) -> np.ndarray:
+    x, px = _c(x, np.float32)
+    w, pw = _c(expert_weight, np.float32)
+    ids, pi = _c(token_expert_idx, np.int32)
+    T, H = x.shape
+    E, _, I = w.shape
+    out = np.zeros((T, I), dtype=np.float64)
+    _check(_lib.oracle_expert_matmul(px, pw, pi, T, H, I, E, _DT[dtype], out.ctypes.data_as(_P)),
+           "expert_matmul")
     return out
 
 

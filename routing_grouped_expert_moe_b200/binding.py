@@ -48,6 +48,10 @@ _SIGS = {
                                _sz, _p, _p, _i]),
     "moe_forward_host": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _p, _sz,
                               _p]),
+    "moe_route_stats_workspace_bytes": (_sz, [_i, _i]),
+    "moe_route_stats": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
+    "moe_expert_matmul_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_expert_matmul": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "moe_get_device_status": (_i, [_p, _p]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
@@ -320,6 +324,49 @@ def forward_host(x_host, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0
                                  ACT[act], _dt(x_host), _ptr(out_host), _ptr(ws), ws.numel(),
                                  _stream()), "moe_forward_host")
     return out_host
+
+
+def route_stats(x, w_gate, gate_bias=None, top_k=2, ws=None):
+    """Router plus its load statistics: returns (topk_idx, topk_gate, expert_counts int32 [E],
+    prob_mean fp32 [E]) and the workspace (for device_status)."""
+    _need(x, "x", dim=2)
+    _need(w_gate, "w_gate", dtype=x.dtype, dim=2)
+    T, H = x.shape
+    E = w_gate.shape[1]
+    if gate_bias is not None:
+        _need(gate_bias, "gate_bias", dtype=torch.float32, dim=1)
+    dev = x.device
+    idx = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    prob = torch.empty(E, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = alloc_workspace(_lib.moe_route_stats_workspace_bytes(T, E), dev)
+    _check(_lib.moe_route_stats(_ptr(x), _ptr(w_gate), _ptr(gate_bias), T, H, E, top_k, _dt(x),
+                                _ptr(idx), _ptr(gate), _ptr(counts), _ptr(prob), _ptr(ws),
+                                ws.numel(), _stream()), "moe_route_stats")
+    return idx, gate, counts, prob, ws
+
+
+def expert_matmul(x, expert_weight, token_expert_idx, out=None, ws=None):
+    """out[t] = x[t] @ expert_weight[token_expert_idx[t]] (one expert per token).
+    Returns (out [T, I], ws)."""
+    _need(x, "x", dim=2)
+    _need(expert_weight, "expert_weight", dtype=x.dtype, dim=3)
+    _need(token_expert_idx, "token_expert_idx", dtype=torch.int32, dim=1)
+    T, H = x.shape
+    E, H2, I = expert_weight.shape
+    if H2 != H or token_expert_idx.shape[0] != T:
+        raise ValueError("shape mismatch between x, expert_weight and token_expert_idx")
+    dev = x.device
+    if out is None:
+        out = torch.empty(T, I, dtype=x.dtype, device=dev)
+    if ws is None:
+        ws = alloc_workspace(_lib.moe_expert_matmul_workspace_bytes(T, H, I, E, _dt(x)), dev)
+    _check(_lib.moe_expert_matmul(_ptr(x), _ptr(expert_weight), _ptr(token_expert_idx), T, H, I, E,
+                                  _dt(x), _ptr(out), _ptr(ws), ws.numel(), _stream()),
+           "moe_expert_matmul")
+    return out, ws
 
 
 def device_status(ws) -> int:

@@ -280,6 +280,129 @@ moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const in
                                     num_sms_current(), as_stream(stream)));
 }
 
+// ---------------------------------------------------------------- router statistics
+// Workspace: [status | logits [T,E] | per-tile counts | per-tile probability sums]
+size_t moe_route_stats_workspace_bytes(int T, int E) {
+  if (T < 0 || E <= 0) return 0;
+  size_t o = align_up(4);
+  o = align_up(o + static_cast<size_t>(T) * E * 4);
+  o = align_up(o + (static_cast<size_t>(T) / 16 + 1) * E * 4);
+  o = align_up(o + (static_cast<size_t>(T) / kStatsBT + 1) * E * 4);
+  return o;
+}
+
+moe_status moe_route_stats(const void* x, const void* w_gate, const float* gate_bias, int T, int H,
+                           int E, int top_k, moe_dtype dt, int32_t* topk_idx, float* topk_gate,
+                           int32_t* expert_counts, float* prob_mean, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (!x || !w_gate || !topk_idx || !topk_gate || !expert_counts || !prob_mean || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, 1, H) || !index_range_ok(T, 1, E)) return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < moe_route_stats_workspace_bytes(T, E)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(expert_counts, 0, E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(cudaMemsetAsync(prob_mean, 0, E * 4, s));
+  }
+  const size_t o_logits = align_up(4);
+  const size_t o_counts = align_up(o_logits + static_cast<size_t>(T) * E * 4);
+  const size_t o_prob = align_up(o_counts + (static_cast<size_t>(T) / 16 + 1) * E * 4);
+  RouteArgs a{};
+  a.x = x; a.wg = w_gate; a.bias = gate_bias;
+  a.T = T; a.H = H; a.E = E; a.top_k = top_k; a.dt_bf16 = dt == MOE_BF16;
+  a.topk_idx = topk_idx; a.topk_gate = topk_gate;
+  a.logits_out = at<float>(ws, o_logits);
+  a.tile_counts = at<int>(ws, o_counts);
+  a.status = at<int>(ws, 0);
+  if (launch_clear_status(a.status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const RoutePlan p = route_plan(T, H, E, a.dt_bf16, num_sms_current(), false);
+  if (launch_route(a, p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_route_stats(a.logits_out, a.tile_counts, p.tiles, T, E,
+                                        at<float>(ws, o_prob), expert_counts, prob_mean, s));
+}
+
+// ---------------------------------------------------------------- k = 1 expert matmul
+// Workspace: [status | tile_counts | counts | offsets | row_token | row_map | x_perm | y]
+namespace {
+struct MatmulWs {
+  size_t tile_counts, counts, offsets, row_token, row_map, x_perm, y, total;
+};
+MatmulWs matmul_ws(int T, int H, int I, int E, moe_dtype dt) {
+  MatmulWs L{};
+  const size_t eb = elem_bytes(dt);
+  size_t o = align_up(4);
+  L.tile_counts = o; o = align_up(o + (static_cast<size_t>(T) / kPermuteBT + 1) * E * 4);
+  L.counts = o;      o = align_up(o + static_cast<size_t>(E) * 4);
+  L.offsets = o;     o = align_up(o + static_cast<size_t>(E + 1) * 4);
+  L.row_token = o;   o = align_up(o + static_cast<size_t>(T) * 4);
+  L.row_map = o;     o = align_up(o + static_cast<size_t>(T) * 4);
+  L.x_perm = o;      o = align_up(o + static_cast<size_t>(T) * H * eb);
+  L.y = o;           o = align_up(o + static_cast<size_t>(T) * I * eb);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+size_t moe_expert_matmul_workspace_bytes(int T, int H, int I, int E, moe_dtype dt) {
+  if (T < 0 || H <= 0 || I <= 0 || E <= 0) return 0;
+  return matmul_ws(T, H, I, E, dt).total;
+}
+
+moe_status moe_expert_matmul(const void* x, const void* expert_weight,
+                             const int32_t* token_expert_idx, int T, int H, int I, int E,
+                             moe_dtype dt, void* out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  moe_status st = check_common(T, H, E, 1, dt);
+  if (st != MOE_OK) return st;
+  if (I <= 0 || I % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !expert_weight || !token_expert_idx || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(expert_weight) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, 1, H) || !index_range_ok(T, 1, I)) return MOE_ERR_UNSUPPORTED;
+  const MatmulWs L = matmul_ws(T, H, I, E, dt);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  int* status = at<int>(ws, 0);
+  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_map = at<int32_t>(ws, L.row_map);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y = at<void>(ws, L.y);
+  // token rearrangement by expert (no capacity limit)
+  PermuteArgs p{};
+  p.idx = token_expert_idx;
+  p.T = T; p.k = 1; p.E = E;
+  p.BT = kPermuteBT;
+  p.tiles = (T + kPermuteBT - 1) / kPermuteBT;
+  p.split = 1;
+  while (p.split < 16 && p.tiles * p.split < 2 * num_sms_current()) p.split *= 2;
+  p.cap = INT32_MAX;
+  p.tile_counts = at<int>(ws, L.tile_counts);
+  p.counts = at<int32_t>(ws, L.counts); p.offsets = offsets;
+  p.row_token = at<int32_t>(ws, L.row_token); p.row_map = row_map;
+  p.x = x; p.x_perm = x_perm; p.H = H; p.elem_bytes = elem_bytes(dt);
+  p.status = status;
+  if (launch_hist(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_scan(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_scatter(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // per-expert matmul of the expert-major rows: y = x_perm W[e]
+  GemmArgs g{};
+  g.offsets = offsets;
+  g.E = E; g.R_max = T; g.T = T; g.status = status;
+  g.N = I; g.K = H; g.out = y;
+  const cudaError_t err =
+      dt == MOE_BF16 ? launch_gemm_tc(2, false, x_perm, T, expert_weight, nullptr, g,
+                                      num_sms_current(), s)
+                     : launch_gemm_simt(2, x_perm, expert_weight, nullptr, g, num_sms_current(), s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  // back to token order: out[t] = y[row_map[t]] (weight 1)
+  return cuda_status(launch_combine(y, nullptr, row_map, T, I, 1, dt == MOE_BF16, out,
+                                    num_sms_current(), s));
+}
+
 }  // extern "C"
 
 namespace {

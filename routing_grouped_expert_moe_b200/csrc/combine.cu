@@ -8,7 +8,8 @@
 // slot order, so the result is the same bit for bit on every run.
 //
 // One warp per token, 16-byte vector loads of each kept row, fp32 accumulation
-// by FMA in slot order, one rounding to the storage type.
+// by FMA in slot order, one rounding to the storage type.  A null gate array
+// means every weight is 1 (the unpermute of a k = 1 matmul: out[t] = y[row]).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,7 +32,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
     for (int s = 0; s < kMaxTopK; ++s) {
       rows[s] = s < k ? __ldg(row_map + static_cast<size_t>(t) * k + s) : -1;
-      g[s] = s < k ? __ldg(gate + static_cast<size_t>(t) * k + s) : 0.f;
+      g[s] = s < k ? (gate ? __ldg(gate + static_cast<size_t>(t) * k + s) : 1.f) : 0.f;
     }
     for (int v = lane; v < nvec; v += 32) {
       float acc[EPV];

@@ -26,6 +26,7 @@
 // owner), warps 2-9 epilogue (TMEM lane quarter = warp % 4; two warps per
 // quarter split the tile's columns, so the activation epilogue of one tile
 // finishes within the next tile's main loop).
+#include <cmath>
 #include <cstdlib>
 
 #include "gemm_common.cuh"
@@ -288,13 +289,27 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const 
 }
 
 // Kernel variant: one CTA per 128-row tile, or CTA pairs sharing 256-row
-// tiles (gemm_tcgen05_pair.cu).  Pairs cut each SM's shared-memory traffic per
-// k-block from 48+48 KB (TMA writes + MMA reads) to 32+32 KB, but round every
-// expert up to 256 rows, so they are chosen when experts hold at least 512
-// rows on average.  MOE_GEMM_VARIANT=1|2 forces one.
+// tiles (gemm_tcgen05_pair.cu).  Pairs cut each SM's operand traffic per
+// k-block from 48 KB to 32 KB, which makes a pair tile ~8% faster than a
+// one-CTA tile of the same rows (measured 0.92-0.94), but round every expert
+// up to 256 rows and run on half as many tile slots.  The host does not know
+// the expert counts (they stay on the device), so it compares the expected
+// number of waves for balanced experts of a = R_max / E rows: an expert of
+// about a rows takes a / BM + 1/2 row tiles on average (its count straddles a
+// tile boundary).  MOE_GEMM_VARIANT=1|2 forces one.
 static int forced_variant() {
   const char* e = getenv("MOE_GEMM_VARIANT");
   return (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
+}
+
+static int choose_variant(int mode, const GemmArgs& g, int num_sms) {
+  const double a = static_cast<double>(g.R_max) / g.E;
+  const double n_tiles = std::ceil(static_cast<double>(g.N) / (mode == 1 ? 128 : 256));
+  const double t1 = g.E * (a / G_BM + 0.5) * n_tiles;
+  const double t2 = g.E * (a / (2 * G_BM) + 0.5) * n_tiles;
+  const double waves1 = std::ceil(t1 / num_sms);
+  const double waves2 = std::ceil(t2 / (num_sms / 2));
+  return 0.92 * waves2 < waves1 ? 2 : 1;
 }
 
 cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
@@ -323,7 +338,7 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
     if (n >= 2 && n < num_sms) num_sms = n;
   }
   int variant = forced_variant();
-  if (variant == 0) variant = (g.R_max >= 512 * g.E) ? 2 : 1;
+  if (variant == 0) variant = choose_variant(mode, g, num_sms);
   if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, mo, ga, num_sms, s);
   switch (mode * 2 + (gather ? 1 : 0)) {
     case 0: return launch_tc<0, false>(ma, mb1, mb3, mo, ga, num_sms, s);

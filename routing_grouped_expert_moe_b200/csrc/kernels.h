@@ -99,6 +99,14 @@ cudaError_t launch_copy_rows(const void* a_src, const GemmArgs& g, int elem_byte
 cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
                            int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- router statistics
+// Per-expert pre-drop counts (summed from the router's per-tile histogram) and
+// the mean over tokens of the full softmax, from fp32 logits [T,E].
+constexpr int kStatsBT = 128;  // tokens per CTA of the probability pass
+cudaError_t launch_route_stats(const float* logits, const int* tile_counts, int count_tiles, int T,
+                               int E, float* tile_prob, int32_t* counts, float* prob_mean,
+                               cudaStream_t s);
+
 // ---------------------------------------------------------------- misc
 // Clears the status word and n counters (the router's tickets).
 cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters = nullptr, int n = 0);

@@ -107,3 +107,24 @@ def test_binding_rejects_int64_indices_and_cpu_tensors():
         B.permute(torch.zeros(4, 2, dtype=torch.int64), 4)
     with pytest.raises(ValueError):
         B.route(torch.zeros(4, 8, dtype=torch.bfloat16), torch.zeros(8, 2, dtype=torch.bfloat16))
+
+
+def test_route_stats_and_expert_matmul_reject_on_host():
+    L = B._lib
+    need = L.moe_route_stats_workspace_bytes(64, 8)
+    assert need >= 64 * 8 * 4 and need % 256 == 0
+    assert L.moe_route_stats_workspace_bytes(-1, 8) == 0
+    args = lambda ws_bytes, prob=FAKE: (FAKE, FAKE, None, 64, 128, 8, 2, 1, FAKE, FAKE, FAKE,  # noqa: E731
+                                        prob, FAKE, ws_bytes, None)
+    assert L.moe_route_stats(*args(need - 1)) == B.ERR_WORKSPACE
+    assert L.moe_route_stats(*args(need, prob=None)) == B.ERR_INVALID_ARG
+    assert L.moe_route_stats(FAKE, FAKE, None, 64, 128, 8, 9, 1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                             need, None) == B.ERR_INVALID_ARG                 # top_k > E
+    mneed = L.moe_expert_matmul_workspace_bytes(64, 128, 256, 8, 1)
+    assert mneed >= 64 * (128 + 256) * 2 and L.moe_expert_matmul_workspace_bytes(64, 128, 0, 8, 1) == 0
+    mm = lambda I=256, ws_bytes=mneed, T=64, w=FAKE: L.moe_expert_matmul(  # noqa: E731
+        FAKE, w, FAKE, T, 128, I, 8, 1, FAKE, FAKE, ws_bytes, None)
+    assert mm(I=100) == B.ERR_INVALID_ARG                                    # I not a multiple of 8
+    assert mm(ws_bytes=mneed - 1) == B.ERR_WORKSPACE
+    assert mm(w=MISALIGNED) == B.ERR_INVALID_ARG
+    assert mm(T=0) == B.OK

@@ -344,3 +344,51 @@ def test_numpy_and_cpp_oracles_agree(act, cf):
     assert a["capacity"] == b["capacity"] and a["dropped"] == b["dropped"]
     np.testing.assert_allclose(b["out"], a["out"], rtol=2.0 ** -7, atol=1e-30)
     assert np.mean(a["out"] == b["out"]) > 0.98
+
+
+# ---------------------------------------------------------------- router load statistics
+
+def test_load_stats_match_library_softmax_and_closed_forms(O):
+    lg = (rng.standard_normal((400, 12)) * 2).astype(np.float32)
+    idx = O.topk_select(lg, 2)
+    st = O.router_load_stats(lg, idx, 12)
+    np.testing.assert_array_equal(st["counts"], np.bincount(idx.ravel(), minlength=12))
+    ref = softmax(lg.astype(np.float64), axis=1).mean(0)            # library softmax
+    np.testing.assert_allclose(st["prob_mean"], ref, rtol=1e-12, atol=0)
+    assert abs(st["prob_mean"].sum() - 1.0) <= 1e-12
+    # equal logits: uniform
+    flat = np.full((7, 5), 0.25, dtype=np.float32)
+    np.testing.assert_allclose(O.router_load_stats(flat, O.topk_select(flat, 1), 5)["prob_mean"],
+                               0.2, rtol=1e-15)
+    # two experts: p_0 is the logistic function of the logit difference
+    two = rng.standard_normal((300, 2)).astype(np.float32)
+    p0 = O.router_load_stats(two, O.topk_select(two, 1), 2)["prob_mean"][0]
+    np.testing.assert_allclose(p0, expit(two[:, 0].astype(np.float64) - two[:, 1]).mean(), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- one expert per token
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_expert_matmul_matches_per_token_library_matmul(O, dtype):
+    T, H, I, E = 50, 24, 40, 5                                      # H != I: a transpose fails
+    x = PY.round_to_bf16(rng.standard_normal((T, H)))
+    w = PY.round_to_bf16(rng.standard_normal((E, H, I)) / 4)
+    ids = rng.integers(0, E, T).astype(np.int32)
+    ids[:3] = 2                                                      # and expert 4 maybe empty
+    got = O.expert_matmul(x, w, ids, dtype)
+    xt, wt = torch.from_numpy(x), torch.from_numpy(w)
+    ref = torch.stack([xt[t] @ wt[int(ids[t])] for t in range(T)])
+    ref = ref.float() if dtype == "f32" else ref.to(torch.bfloat16)
+    np.testing.assert_allclose(got, ref.double().numpy(), rtol=2.0 ** -7 if dtype == "bf16" else 1e-6,
+                               atol=0)
+    assert np.mean(got == ref.double().numpy()) > 0.97
+
+
+def test_expert_matmul_one_expert_is_dense_and_ids_are_checked(O):
+    x = rng.standard_normal((9, 16)).astype(np.float32).astype(np.float64)
+    w = rng.standard_normal((1, 16, 8)).astype(np.float32).astype(np.float64)
+    got = O.expert_matmul(x, w, np.zeros(9, dtype=np.int32), "f32")
+    np.testing.assert_allclose(got, (torch.from_numpy(x) @ torch.from_numpy(w[0])).float().numpy(),
+                               rtol=1e-6)
+    with pytest.raises(O.IndexOutOfRange):
+        O.expert_matmul(x, w, np.array([0] * 8 + [1], dtype=np.int32), "f32")
