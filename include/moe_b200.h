@@ -219,6 +219,37 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
                              moe_dtype dt, void* out, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
 
+/* Threshold gating (a variable number of experts per token).  [P2] §3.2.1:
+ * compute every expert's gate score (softmax over all E of the logits, §2.1),
+ * keep only the experts whose score exceeds delta (default 1/E), renormalise
+ * the kept ones.  Readings where the page is silent: kept experts are ordered
+ * largest first (ties to the lower id); at most k_max are kept (1 <= k_max <=
+ * min(8, E), the caller's slot count); when none exceeds delta the largest
+ * alone is kept.  delta <= 0 selects the default 1/E.
+ *   topk_idx [T,k_max]: kept ids, then -1;  topk_gate [T,k_max]: renormalised
+ *   gates exp(l_s - l_0) / sum_kept exp(l_j - l_0), then 0;
+ *   n_selected [T]: number kept;  token_offsets [T+1] (nullable): exclusive
+ *   prefix sum of n_selected, the CSR row offsets of the selection.
+ * moe_threshold_select starts from caller-given fp32 logits [T,E] (parity
+ * hook, like moe_route_from_logits).                                        */
+moe_status moe_threshold_select(const float* logits, int T, int E, int k_max, float delta,
+                                int32_t* topk_idx, float* topk_gate, int32_t* n_selected,
+                                int32_t* token_offsets, moe_stream_t stream);
+
+/* The whole layer with threshold gating: router logits -> threshold selection
+ * (as above) -> permute (slots with id -1 are unused, not errors; capacity
+ * C = ceil(capacity_factor * T * k_max / E)) -> grouped FFN -> combine over
+ * each token's kept slots.  topk_idx_out [T,k_max] and n_selected_out [T] may
+ * be NULL.  ws: at least moe_forward_threshold_workspace_bytes(...) bytes.   */
+size_t moe_forward_threshold_workspace_bytes(int T, int H, int F, int E, int k_max, moe_act act,
+                                             moe_dtype dt);
+moe_status moe_forward_threshold(const void* x, const void* w_gate, const float* gate_bias,
+                                 const void* w1, const void* w3, const void* w2,
+                                 int T, int H, int F, int E, int k_max, float delta,
+                                 float capacity_factor, moe_act act, moe_dtype dt, void* out,
+                                 int32_t* topk_idx_out, int32_t* n_selected_out,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the status the kernels of the last
  * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */
 moe_status moe_get_device_status(void* ws, moe_stream_t stream);

@@ -153,6 +153,45 @@ int oracle_topk_gates_literal(const float* logits, const int32_t* idx, int T, in
   return 0;
 }
 
+// Threshold gating: p = softmax over all E (float64, NaN logits carry no mass);
+// keep the experts with p > delta, largest first (ties to the lower id), at most
+// k_max, the largest always; g_s = exp(l_s - l_0) / sum_kept exp(l_j - l_0).
+// delta <= 0: 1/E (as float32).  idx/gate padded with -1 / 0.
+int oracle_threshold_select(const float* logits, int T, int E, int k_max, float delta,
+                            int32_t* idx, float* gate, int32_t* n_sel) {
+  if (k_max < 1 || k_max > E || k_max > 64) return 1;
+  const double d = delta > 0.0f ? static_cast<double>(delta)
+                                : static_cast<double>(1.0f / static_cast<float>(E));
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + static_cast<int64_t>(t) * E;
+    std::vector<int> order;  // insertion into descending order, as oracle_topk_select
+    for (int e = 0; e < E; ++e) {
+      size_t pos = order.size();
+      while (pos > 0 && ranks_before(l[e], e, l[order[pos - 1]], order[pos - 1])) --pos;
+      order.insert(order.begin() + pos, e);
+    }
+    double mx = -INFINITY;
+    for (int e = 0; e < E; ++e)
+      if (!std::isnan(l[e])) mx = std::fmax(mx, static_cast<double>(l[e]));
+    double den = 0.0;
+    for (int e = 0; e < E; ++e)
+      if (!std::isnan(l[e])) den += std::exp(static_cast<double>(l[e]) - mx);
+    int n = 1;
+    while (n < k_max && std::exp(static_cast<double>(l[order[n]]) - mx) / den > d) ++n;
+    double z[64], zs = 0.0;
+    for (int s = 0; s < n; ++s) {
+      z[s] = std::exp(static_cast<double>(l[order[s]]) - static_cast<double>(l[order[0]]));
+      zs += z[s];
+    }
+    for (int s = 0; s < k_max; ++s) {
+      idx[static_cast<int64_t>(t) * k_max + s] = s < n ? order[s] : -1;
+      gate[static_cast<int64_t>(t) * k_max + s] = s < n ? static_cast<float>(z[s] / zs) : 0.0f;
+    }
+    n_sel[t] = n;
+  }
+  return 0;
+}
+
 // C = ceil(cf * T * k / E), exact for the float32 cf (cf = m * 2^x with integer m);
 // *cap = -1 when cf <= 0 (no limit).
 int oracle_capacity(float cf, int T, int k, int E, int64_t* cap) {
@@ -187,17 +226,19 @@ int oracle_capacity(float cf, int T, int k, int E, int64_t* cap) {
 
 // Stable, capacity-limited permutation of (token, slot) pairs into expert-major
 // rows, first come first kept (t ascending, then s).  cap < 0: no limit.
-int oracle_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int64_t* counts,
-                   int64_t* kept, int64_t* offsets, int64_t* row_token, int64_t* row_slot,
-                   int64_t* row_map, int64_t* R_out) {
+// empty_slots: id -1 marks an unused slot (threshold gating), skipped silently.
+int oracle_permute(const int32_t* idx, int T, int k, int E, int64_t cap, int empty_slots,
+                   int64_t* counts, int64_t* kept, int64_t* offsets, int64_t* row_token,
+                   int64_t* row_slot, int64_t* row_map, int64_t* R_out) {
   const int64_t n = static_cast<int64_t>(T) * k;
   for (int64_t i = 0; i < n; ++i)
-    if (idx[i] < 0 || idx[i] >= E) return 2;
+    if ((idx[i] < 0 || idx[i] >= E) && !(empty_slots && idx[i] == -1)) return 2;
   const int64_t limit = cap < 0 ? n : cap;
   std::vector<int64_t> arrival(n, -1);
   for (int e = 0; e < E; ++e) { counts[e] = 0; kept[e] = 0; }
   for (int64_t i = 0; i < n; ++i) {
     const int e = idx[i];
+    if (e == -1) continue;
     counts[e] += 1;
     if (kept[e] < limit) arrival[i] = kept[e]++;
   }

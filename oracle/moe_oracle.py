@@ -173,13 +173,19 @@ class IndexOutOfRange(ValueError):
     """An expert id outside [0, E): an error, never clamped ([P4] §5.2, §7)."""
 
 
-def expert_counts(idx, E: int) -> np.ndarray:
-    """count[e] = number of (token, slot) pairs routed to expert e."""
+def expert_counts(idx, E: int, empty_slots: bool = False) -> np.ndarray:
+    """count[e] = number of (token, slot) pairs routed to expert e.
+
+    With empty_slots, id -1 marks an unused slot (threshold gating) and is skipped.
+    """
     idx = np.asarray(idx)
-    if idx.size and (idx.min() < 0 or idx.max() >= E):
+    flat = idx.reshape(-1)
+    if empty_slots:
+        flat = flat[flat != -1]
+    if flat.size and (flat.min() < 0 or flat.max() >= E):
         raise IndexOutOfRange("expert id outside [0, E)")
     c = np.zeros(E, dtype=np.int64)
-    for e in idx.reshape(-1):
+    for e in flat:
         c[int(e)] += 1
     return c
 
@@ -198,7 +204,7 @@ def capacity(capacity_factor: float, T: int, k: int, E: int):
     return int(math.ceil(q))
 
 
-def permute(idx, E: int, cap=None) -> dict:
+def permute(idx, E: int, cap=None, empty_slots: bool = False) -> dict:
     """Stable, capacity-limited permutation of (token, slot) pairs into expert-major rows.
 
     Walk tokens t = 0..T-1 and, within a token, slots s = 0..k-1.  The pair
@@ -209,17 +215,21 @@ def permute(idx, E: int, cap=None) -> dict:
     token order within an expert).
 
     Returns counts (pre-drop), kept, offsets[E+1], row_token[R], row_slot[R],
-    row_map[T,k] (row index or -1 when dropped) and the number dropped.
+    row_map[T,k] (row index or -1 when dropped) and the number dropped.  With
+    empty_slots, slots holding id -1 are unused: not counted, not dropped,
+    row_map -1 (threshold gating leaves a token's trailing slots empty).
     """
     idx = np.asarray(idx)
     T, k = idx.shape
-    counts = expert_counts(idx, E)
+    counts = expert_counts(idx, E, empty_slots)
     limit = cap if cap is not None else T * k
     kept = np.zeros(E, dtype=np.int64)
     arrival = np.full((T, k), -1, dtype=np.int64)
     for t in range(T):
         for s in range(k):
             e = int(idx[t, s])
+            if e == -1 and empty_slots:
+                continue
             if kept[e] < limit:
                 arrival[t, s] = kept[e]
                 kept[e] += 1
@@ -237,8 +247,9 @@ def permute(idx, E: int, cap=None) -> dict:
                 row_token[r] = t
                 row_slot[r] = s
                 row_map[t, s] = r
+    used = int(counts.sum())
     return {"counts": counts, "kept": kept, "offsets": offsets, "row_token": row_token,
-            "row_slot": row_slot, "row_map": row_map, "dropped": int(T * k - R), "R": R}
+            "row_slot": row_slot, "row_map": row_map, "dropped": int(used - R), "R": R}
 
 
 # --------------------------------------------------------------------------
@@ -319,6 +330,61 @@ def combine(y, gates, row_map, dtype: str) -> np.ndarray:
         m = r >= 0
         out[m] += g[m, s][:, None] * y[r[m]]
     return round_to(dtype, out)
+
+
+# --------------------------------------------------------------------------
+# Threshold gating.   [P2] §3.2.1: compute all experts' gate scores, keep the
+# experts whose score exceeds delta (default 1/E), renormalise the kept ones.
+# --------------------------------------------------------------------------
+
+
+def threshold_select(logits, k_max: int, delta=None) -> dict:
+    """Per token: p = softmax over all E (float64); keep the experts with p > delta,
+    largest first (ties to the lower id), at most k_max; when none exceeds delta
+    the largest alone is kept.  Gates g_s = exp(l_s - l_0) / sum_kept exp(l_j - l_0).
+    delta None or <= 0: the default 1/E (as the float32 the library uses).
+    Returns idx [T,k_max] (-1 pads), gate [T,k_max] fp32 (0 pads), n_sel [T]."""
+    lg = np.asarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    if not 1 <= k_max <= E:
+        raise ValueError("k_max must lie in [1, E]")
+    d = float(np.float32(1.0 / E)) if delta is None or delta <= 0 else float(np.float32(delta))
+    idx = np.full((T, k_max), -1, dtype=np.int32)
+    gate = np.zeros((T, k_max), dtype=np.float32)
+    n_sel = np.zeros(T, dtype=np.int32)
+    for t in range(T):
+        row = [float(v) for v in lg[t]]
+        order = sorted(range(E), key=lambda e: (_rank_key(row[e]), e))
+        l64 = np.asarray(row, dtype=np.float64)
+        z = np.exp(l64 - np.nanmax(l64))
+        p = z / np.nansum(z)
+        kept = [order[0]]
+        for e in order[1:k_max]:
+            if not p[e] > d:
+                break
+            kept.append(e)
+        zk = np.exp(l64[kept] - l64[kept[0]])
+        n_sel[t] = len(kept)
+        idx[t, :len(kept)] = kept
+        gate[t, :len(kept)] = (zk / zk.sum()).astype(np.float32)
+    return {"topk_idx": idx, "topk_gate": gate, "n_sel": n_sel}
+
+
+def moe_forward_threshold(x, w_gate, gate_bias, w1, w3, w2, k_max: int, delta,
+                          capacity_factor: float, act: str, dtype: str, logits=None) -> dict:
+    """The layer with threshold gating: unused slots (-1) carry no row; capacity
+    C = ceil(cf * T * k_max / E)."""
+    x = np.asarray(x)
+    T = x.shape[0]
+    if logits is None:
+        logits = router_logits(x, w_gate, gate_bias)
+    E = logits.shape[1]
+    sel = threshold_select(logits, k_max, delta)
+    cap = capacity(capacity_factor, T, k_max, E)
+    perm = permute(sel["topk_idx"], E, cap, empty_slots=True)
+    y = grouped_ffn(x, perm, w1, w3, w2, act, dtype, E)
+    out = combine(y, sel["topk_gate"], perm["row_map"], dtype)
+    return {"logits": logits, **sel, "capacity": cap, "y": y, "out": out, **perm}
 
 
 # --------------------------------------------------------------------------

@@ -40,7 +40,8 @@ for _name, _args in {
     "oracle_topk_gates": [_P, _P, _I, _I, _I, _P],
     "oracle_topk_gates_literal": [_P, _P, _I, _I, _I, _P],
     "oracle_capacity": [ctypes.c_float, _I, _I, _I, _P],
-    "oracle_permute": [_P, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, _P],
+    "oracle_permute": [_P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _P],
+    "oracle_threshold_select": [_P, _I, _I, _I, ctypes.c_float, _P, _P, _P],
     "oracle_grouped_ffn": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P],
     "oracle_combine": [_P, _I, _P, _P, _I, _I, _I, _P],
     "oracle_activation": [_P, _I64, _I, _P],
@@ -147,7 +148,7 @@ def capacity(capacity_factor: float, T: int, k: int, E: int):
     return None if cap[0] < 0 else int(cap[0])
 
 
-def permute(idx, E: int, cap=None) -> dict:
+def permute(idx, E: int, cap=None, empty_slots: bool = False) -> dict:
     ix, pi = _c(idx, np.int32)
     T, k = ix.shape
     n = T * k
@@ -159,15 +160,47 @@ def permute(idx, E: int, cap=None) -> dict:
     row_map = np.full((T, k), -1, dtype=np.int64)
     R = np.zeros(1, dtype=np.int64)
     p = lambda a: a.ctypes.data_as(_P)  # noqa: E731
-    _check(_lib.oracle_permute(pi, T, k, E, -1 if cap is None else int(cap), p(counts), p(kept),
-                               p(offsets), p(row_token), p(row_slot), p(row_map), p(R)), "permute")
+    _check(_lib.oracle_permute(pi, T, k, E, -1 if cap is None else int(cap), int(empty_slots),
+                               p(counts), p(kept), p(offsets), p(row_token), p(row_slot),
+                               p(row_map), p(R)), "permute")
     R = int(R[0])
     return {"counts": counts, "kept": kept, "offsets": offsets, "row_token": row_token[:R].copy(),
-            "row_slot": row_slot[:R].copy(), "row_map": row_map, "dropped": int(n - R), "R": R}
+            "row_slot": row_slot[:R].copy(), "row_map": row_map,
+            "dropped": int(counts.sum() - R), "R": R}
 
 
-def expert_counts(idx, E: int) -> np.ndarray:
-    return permute(idx, E)["counts"]
+def expert_counts(idx, E: int, empty_slots: bool = False) -> np.ndarray:
+    return permute(idx, E, None, empty_slots)["counts"]
+
+
+def threshold_select(logits, k_max: int, delta=None) -> dict:
+    lg, pl = _c(logits, np.float32)
+    T, E = lg.shape
+    if not 1 <= k_max <= E:
+        raise ValueError("k_max must lie in [1, E]")
+    idx = np.empty((T, k_max), dtype=np.int32)
+    gate = np.empty((T, k_max), dtype=np.float32)
+    n_sel = np.empty(T, dtype=np.int32)
+    d = 0.0 if delta is None else float(delta)
+    p = lambda a: a.ctypes.data_as(_P)  # noqa: E731
+    _check(_lib.oracle_threshold_select(pl, T, E, k_max, ctypes.c_float(d), p(idx), p(gate),
+                                        p(n_sel)), "threshold_select")
+    return {"topk_idx": idx, "topk_gate": gate, "n_sel": n_sel}
+
+
+def moe_forward_threshold(x, w_gate, gate_bias, w1, w3, w2, k_max: int, delta,
+                          capacity_factor: float, act: str, dtype: str, logits=None) -> dict:
+    x = np.asarray(x)
+    T = x.shape[0]
+    if logits is None:
+        logits = router_logits(x, w_gate, gate_bias)
+    E = logits.shape[1]
+    sel = threshold_select(logits, k_max, delta)
+    cap = capacity(capacity_factor, T, k_max, E)
+    perm = permute(sel["topk_idx"], E, cap, empty_slots=True)
+    y = grouped_ffn(x, perm, w1, w3, w2, act, dtype, E)
+    out = combine(y, sel["topk_gate"], perm["row_map"], dtype)
+    return {"logits": logits, **sel, "capacity": cap, "y": y, "out": out, **perm}
 
 
 def _activation(z, which: int) -> np.ndarray:

@@ -52,6 +52,10 @@ _SIGS = {
     "moe_route_stats": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_expert_matmul_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "moe_expert_matmul": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "moe_threshold_select": (_i, [_p, _i, _i, _i, _f, _p, _p, _p, _p, _p]),
+    "moe_forward_threshold_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "moe_forward_threshold": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _i, _i, _p,
+                                   _p, _p, _p, _sz, _p]),
     "moe_get_device_status": (_i, [_p, _p]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
@@ -366,6 +370,42 @@ def expert_matmul(x, expert_weight, token_expert_idx, out=None, ws=None):
     _check(_lib.moe_expert_matmul(_ptr(x), _ptr(expert_weight), _ptr(token_expert_idx), T, H, I, E,
                                   _dt(x), _ptr(out), _ptr(ws), ws.numel(), _stream()),
            "moe_expert_matmul")
+    return out, ws
+
+
+def threshold_select(logits, k_max, delta=0.0, token_offsets=False):
+    """Threshold gating from fp32 logits: (idx [T,k_max] (-1 pads), gate [T,k_max],
+    n_selected [T][, token_offsets [T+1]])."""
+    _need(logits, "logits", dtype=torch.float32, dim=2)
+    T, E = logits.shape
+    dev = logits.device
+    idx = torch.empty(T, k_max, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, k_max, dtype=torch.float32, device=dev)
+    n = torch.empty(T, dtype=torch.int32, device=dev)
+    offs = torch.empty(T + 1, dtype=torch.int32, device=dev) if token_offsets else None
+    _check(_lib.moe_threshold_select(_ptr(logits), T, E, k_max, ctypes.c_float(delta), _ptr(idx),
+                                     _ptr(gate), _ptr(n), _ptr(offs), _stream()),
+           "moe_threshold_select")
+    return (idx, gate, n, offs) if token_offsets else (idx, gate, n)
+
+
+def forward_threshold(x, w_gate, gate_bias, w1, w3, w2, k_max, delta=0.0, capacity_factor=0.0,
+                      act="swiglu", out=None, ws=None, topk_idx_out=None, n_selected_out=None):
+    """The layer with threshold gating; returns (out, ws)."""
+    _need(x, "x", dim=2)
+    T, H = x.shape
+    E = w_gate.shape[1]
+    F = 8 if act == "identity" else w1.shape[2]
+    if out is None:
+        out = torch.empty_like(x)
+    if ws is None:
+        ws = alloc_workspace(_lib.moe_forward_threshold_workspace_bytes(T, H, F, E, k_max, ACT[act],
+                                                                         _dt(x)), x.device)
+    _check(_lib.moe_forward_threshold(_ptr(x), _ptr(w_gate), _ptr(gate_bias), _ptr(w1), _ptr(w3),
+                                      _ptr(w2), T, H, F, E, k_max, ctypes.c_float(delta),
+                                      ctypes.c_float(capacity_factor), ACT[act], _dt(x), _ptr(out),
+                                      _ptr(topk_idx_out), _ptr(n_selected_out), _ptr(ws),
+                                      ws.numel(), _stream()), "moe_forward_threshold")
     return out, ws
 
 

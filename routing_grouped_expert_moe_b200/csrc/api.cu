@@ -39,10 +39,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 //             counts | offsets | row_token | row_map | x_perm | h | y | x_stage | out_stage]
 struct WsLayout {
   size_t status, topk_idx, topk_gate, tile_counts, tickets, partials, counts, offsets, row_token,
-      row_map, x_perm, h, y, x_stage, out_stage, total;
+      row_map, x_perm, h, y, x_stage, out_stage, logits, n_sel, total;
 };
 
-WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt, bool host_stage) {
+WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt, bool host_stage,
+                   bool threshold = false) {
   WsLayout L{};
   const size_t eb = elem_bytes(dt);
   const size_t R = static_cast<size_t>(T) * k;
@@ -64,6 +65,10 @@ WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt,
   if (host_stage) {
     L.x_stage = o;   o = align_up(o + static_cast<size_t>(T) * H * eb);
     L.out_stage = o; o = align_up(o + static_cast<size_t>(T) * H * eb);
+  }
+  if (threshold) {
+    L.logits = o;    o = align_up(o + static_cast<size_t>(T) * E * 4);
+    L.n_sel = o;     o = align_up(o + (static_cast<size_t>(T) + 1) * 4);
   }
   L.total = o;
   return L;
@@ -407,11 +412,20 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
 
 namespace {
 
+// Threshold gating instead of top-k (moe_forward_threshold): top_k is then the
+// slot count k_max and delta the probability threshold.
+struct Gating {
+  bool threshold = false;
+  float delta = 0.f;
+  int32_t* n_sel_out = nullptr;
+};
+
 moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bias, const void* w1,
                         const void* w3, const void* w2, int T, int H, int F, int E, int top_k,
                         float capacity_factor, moe_act act, moe_dtype dt, void* out,
                         int32_t* topk_idx_out, int32_t* expert_counts_out, void* ws,
-                        size_t ws_bytes, moe_stream_t stream, cudaEvent_t const* ev) {
+                        size_t ws_bytes, moe_stream_t stream, cudaEvent_t const* ev,
+                        const Gating& gating = Gating()) {
   moe_status st = check_common(T, H, E, top_k, dt);
   if (st != MOE_OK) return st;
   if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU && act != MOE_ACT_IDENTITY)
@@ -426,7 +440,7 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   }
   if (!index_range_ok(T, top_k, H > F ? H : F) || !index_range_ok(T, 1, E))
     return MOE_ERR_UNSUPPORTED;
-  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false);
+  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false, gating.threshold);
   if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
 
@@ -459,23 +473,37 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   ra.status = status;
   ra.partials = at<float>(ws, L.partials);
   ra.tickets = tickets;
+  if (gating.threshold) {  // the router's logits feed the threshold selection
+    ra.logits_out = at<float>(ws, L.logits);
+    ra.tile_counts = nullptr;
+  }
   const RoutePlan rp = route_plan(T, H, E, bf16, nsm, true);
   if (launch_route(ra, rp, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (mark(1) != cudaSuccess) return MOE_ERR_CUDA;
-  // 2. scan + scatter over the router's token tiles
   PermuteArgs pa{};
   pa.idx = topk_idx;
   pa.T = T; pa.k = top_k; pa.E = E;
   pa.BT = rp.BT; pa.tiles = rp.tiles;
+  pa.tile_counts = at<int>(ws, L.tile_counts);
+  pa.status = status;
+  if (gating.threshold) {
+    int32_t* n_sel = gating.n_sel_out ? gating.n_sel_out : at<int32_t>(ws, L.n_sel);
+    if (launch_route_threshold(ra.logits_out, T, E, top_k, gating.delta, topk_idx, topk_gate,
+                               n_sel, nullptr, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    pa.BT = kPermuteBT;
+    pa.tiles = (T + kPermuteBT - 1) / kPermuteBT;
+    pa.empty_slots = 1;
+    if (launch_hist(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (mark(1) != cudaSuccess) return MOE_ERR_CUDA;
+  // 2. scan + scatter over the router's (or the histogram's) token tiles
   // enough scatter CTAs to keep the x_perm row copies near HBM bandwidth
   pa.split = 1;
   if (x_perm)
     while (pa.split < 16 && pa.tiles * pa.split < 2 * nsm) pa.split *= 2;
   pa.cap = capacity_of(capacity_factor, T, top_k, E);
-  pa.tile_counts = ra.tile_counts;
   pa.counts = counts; pa.offsets = offsets; pa.row_token = row_token; pa.row_map = row_map;
   pa.x = x; pa.x_perm = x_perm; pa.H = H; pa.elem_bytes = elem_bytes(dt);
-  pa.status = status;
   if (launch_scan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (mark(2) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_scatter(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -504,6 +532,43 @@ moe_status moe_forward(const void* x, const void* w_gate, const float* gate_bias
                        size_t ws_bytes, moe_stream_t stream) {
   return forward_impl(x, w_gate, gate_bias, w1, w3, w2, T, H, F, E, top_k, capacity_factor, act,
                       dt, out, topk_idx_out, expert_counts_out, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_threshold_select(const float* logits, int T, int E, int k_max, float delta,
+                                int32_t* topk_idx, float* topk_gate, int32_t* n_selected,
+                                int32_t* token_offsets, moe_stream_t stream) {
+  if (T < 0 || E <= 0 || k_max <= 0 || k_max > E) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || k_max > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (!(delta == delta)) return MOE_ERR_INVALID_ARG;  // NaN
+  if (!logits || !topk_idx || !topk_gate || !n_selected) return MOE_ERR_INVALID_ARG;
+  if (!index_range_ok(T, 1, E)) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0)
+    return cuda_status(token_offsets ? cudaMemsetAsync(token_offsets, 0, 4, s) : cudaSuccess);
+  const float d = delta > 0.f ? delta : 1.f / static_cast<float>(E);
+  return cuda_status(launch_route_threshold(logits, T, E, k_max, d, topk_idx, topk_gate,
+                                            n_selected, token_offsets, s));
+}
+
+size_t moe_forward_threshold_workspace_bytes(int T, int H, int F, int E, int k_max, moe_act act,
+                                             moe_dtype dt) {
+  if (T < 0 || H <= 0 || F <= 0 || E <= 0 || k_max <= 0) return 0;
+  return ws_layout(T, H, F, E, k_max, act, dt, false, true).total;
+}
+
+moe_status moe_forward_threshold(const void* x, const void* w_gate, const float* gate_bias,
+                                 const void* w1, const void* w3, const void* w2, int T, int H,
+                                 int F, int E, int k_max, float delta, float capacity_factor,
+                                 moe_act act, moe_dtype dt, void* out, int32_t* topk_idx_out,
+                                 int32_t* n_selected_out, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  if (!(delta == delta)) return MOE_ERR_INVALID_ARG;
+  Gating g;
+  g.threshold = true;
+  g.delta = delta > 0.f ? delta : (E > 0 ? 1.f / static_cast<float>(E) : 0.f);
+  g.n_sel_out = n_selected_out;
+  return forward_impl(x, w_gate, gate_bias, w1, w3, w2, T, H, F, E, k_max, capacity_factor, act,
+                      dt, out, topk_idx_out, nullptr, ws, ws_bytes, stream, nullptr, g);
 }
 
 moe_status moe_forward_timed(const void* x, const void* w_gate, const float* gate_bias,

@@ -56,6 +56,7 @@ struct PermuteArgs {
   void* x_perm;         // [T*k,H] or null
   int H, elem_bytes;
   int* status;
+  int empty_slots;      // 1: id -1 marks an unused slot (threshold gating), not an error
 };
 
 constexpr int kPermuteBT = 128;
@@ -106,6 +107,14 @@ constexpr int kStatsBT = 128;  // tokens per CTA of the probability pass
 cudaError_t launch_route_stats(const float* logits, const int* tile_counts, int count_tiles, int T,
                                int E, float* tile_prob, int32_t* counts, float* prob_mean,
                                cudaStream_t s);
+
+// ---------------------------------------------------------------- threshold gating
+// Per token: experts with softmax probability > delta, largest first, at most
+// k_max (the largest always kept); idx/gate [T,k_max] padded with -1 / 0;
+// n_sel [T]; token_offsets [T+1] (exclusive prefix of n_sel) when non-null.
+cudaError_t launch_route_threshold(const float* logits, int T, int E, int k_max, float delta,
+                                   int32_t* idx, float* gate, int32_t* n_sel,
+                                   int32_t* token_offsets, cudaStream_t s);
 
 // ---------------------------------------------------------------- misc
 // Clears the status word and n counters (the router's tickets).

@@ -23,7 +23,8 @@ namespace moe {
 constexpr int kPermThreads = 256;
 
 // Per-tile expert histogram of caller-given ids (the fused path gets it from
-// the router).  Out-of-range ids are reported and not counted.
+// the router).  Out-of-range ids are reported and not counted; with
+// empty_slots, id -1 is an unused slot and is skipped silently.
 __global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
   __shared__ int cnt_s[kMaxE];
   const int lane = threadIdx.x & 31;
@@ -37,7 +38,7 @@ __global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
     if (i < a1) {
       e = a.idx[i];
       if (e < 0 || e >= a.E) {
-        record_status(a.status, kStatusIndexOutOfRange);
+        if (!(a.empty_slots && e == -1)) record_status(a.status, kStatusIndexOutOfRange);
         e = -1;
       }
     }

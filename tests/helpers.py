@@ -52,6 +52,32 @@ def gapped_inputs(cfg: synth.MoEConfig, with_weights: bool = True, max_rounds: i
     return d
 
 
+def threshold_margin_violations(logits: np.ndarray, delta: float, rel: float = 1e-3) -> np.ndarray:
+    """Tokens with an expert whose softmax probability lies within rel * delta of
+    delta: there a float32 and a float64 evaluation could decide differently."""
+    lg = logits.astype(np.float64)
+    z = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    return np.nonzero(np.any(np.abs(p - delta) < rel * delta, axis=1))[0]
+
+
+def threshold_inputs(cfg: synth.MoEConfig, delta: float, k_max: int, max_rounds: int = 50) -> dict:
+    """gapped_inputs whose tokens also keep every probability away from delta and
+    a 1e-3 gap between each of their k_max + 1 largest logits."""
+    d = gapped_inputs(cfg)
+    x = d["x"]
+    wg = as_np(d["w_gate"])
+    b = None if d["gate_bias"] is None else as_np(d["gate_bias"])
+    for attempt in range(max_rounds):
+        lg = O.router_logits(as_np(x), wg, b)
+        bad = np.union1d(threshold_margin_violations(lg, delta), gap_violations(lg, k_max))
+        if len(bad) == 0:
+            d["x"] = x
+            return d
+        x[torch.from_numpy(bad)] = synth.redraw_rows(cfg, len(bad), 100 + attempt)
+    raise RuntimeError("threshold margin enforcement did not converge")
+
+
 def rel_err(gpu, ref) -> float:
     g = np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)

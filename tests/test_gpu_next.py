@@ -1,6 +1,7 @@
 """Parity of the rows built past the layer itself: the router's load statistics
-(moe_route_stats) and the one-expert-per-token matmul (moe_expert_matmul),
-each against both CPU oracles."""
+(moe_route_stats), the one-expert-per-token matmul (moe_expert_matmul) and
+threshold gating (moe_threshold_select, moe_forward_threshold), each against
+both CPU oracles."""
 from dataclasses import replace
 
 import numpy as np
@@ -110,3 +111,59 @@ def test_expert_matmul_bad_id_gives_zero_row_and_status():
     keep = np.setdiff1d(np.arange(T), [5, 9])
     ref = O.expert_matmul(as_np(x[torch.from_numpy(keep)]), as_np(w), ids.numpy()[keep], "bf16")
     assert rel_err(got[keep], ref) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------- threshold gating
+
+@pytest.mark.parametrize("E,k_max", [(8, 4), (32, 8), (128, 8), (5, 5)])
+def test_threshold_select_from_logits(E, k_max):
+    from tests.helpers import threshold_margin_violations
+    T = 3000
+    delta = float(np.float32(1.0 / E))
+    lg = synth.random_logits(5000 + E, T, E, scale=2.0).numpy()
+    for attempt in range(20):                         # keep probabilities away from delta
+        bad = threshold_margin_violations(lg, delta)
+        if len(bad) == 0:
+            break
+        lg[bad] = synth.random_logits(5100 + attempt, len(bad), E, scale=2.0).numpy()
+    assert len(threshold_margin_violations(lg, delta)) == 0
+    idx, gate, n, offs = B().threshold_select(torch.from_numpy(lg).cuda(), k_max, token_offsets=True)
+    for orc in (O, OC):
+        ref = orc.threshold_select(lg, k_max)
+        np.testing.assert_array_equal(as_np(idx), ref["topk_idx"])
+        np.testing.assert_array_equal(as_np(n), ref["n_sel"])
+        assert np.max(np.abs(as_np(gate) - ref["topk_gate"])) <= 1e-6
+    np.testing.assert_array_equal(as_np(offs), np.concatenate([[0], np.cumsum(as_np(n))]))
+    assert 1 <= as_np(n).min() and as_np(n).max() <= k_max
+
+
+THR_CFGS = [
+    (replace(synth.CONFIGS["mixtral_e8"], name="thr_e8", T=400, H=256, F=384, seed=6001), 4, 0.0),
+    (replace(synth.CONFIGS["e32_long"], name="thr_e32", T=600, H=128, F=136, seed=6002), 8, 0.0),
+    (replace(synth.CONFIGS["page1_gelu"], name="thr_gelu_cap", T=512, H=256, F=256, seed=6003), 3,
+     0.9),
+    (synth.CONFIGS["tiny_f32"], 3, 0.0),
+]
+
+
+@pytest.mark.parametrize("cfg,k_max,cf", THR_CFGS, ids=lambda c: getattr(c, "name", str(c)))
+def test_forward_threshold(cfg, k_max, cf):
+    from tests.helpers import threshold_inputs
+    delta = float(np.float32(1.0 / cfg.E))
+    d = threshold_inputs(cfg, delta, k_max)
+    g = {k: (None if v is None else v.cuda()) for k, v in d.items()}
+    idx = torch.empty(cfg.T, k_max, dtype=torch.int32, device="cuda")
+    n = torch.empty(cfg.T, dtype=torch.int32, device="cuda")
+    out, ws = B().forward_threshold(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"],
+                                    k_max, 0.0, cf, cfg.act, topk_idx_out=idx, n_selected_out=n)
+    assert B().device_status(ws) == B().OK
+    f = lambda t: None if t is None else as_np(t)  # noqa: E731
+    for orc in (O, OC):
+        ref = orc.moe_forward_threshold(f(d["x"]), f(d["w_gate"]), f(d["gate_bias"]), f(d["w1"]),
+                                        f(d["w3"]), f(d["w2"]), k_max, None, cf, cfg.act, cfg.dtype)
+        np.testing.assert_array_equal(as_np(idx), ref["topk_idx"])
+        np.testing.assert_array_equal(as_np(n), ref["n_sel"])
+        err = rel_err(as_np(out), ref["out"])
+        assert err <= TOL[cfg.dtype], err
+    nn = as_np(n)
+    assert nn.min() >= 1 and (nn.max() > 1 or k_max == 1)

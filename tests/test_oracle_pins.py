@@ -392,3 +392,73 @@ def test_expert_matmul_one_expert_is_dense_and_ids_are_checked(O):
                                rtol=1e-6)
     with pytest.raises(O.IndexOutOfRange):
         O.expert_matmul(x, w, np.array([0] * 8 + [1], dtype=np.int32), "f32")
+
+
+# ---------------------------------------------------------------- threshold gating
+
+def _threshold_reference(lg, k_max, delta):
+    """The definition written with library calls: softmax (scipy), a stable sort
+    by descending logit, the prefix of experts above delta (at least one)."""
+    p = softmax(lg.astype(np.float64), axis=1)
+    T, E = lg.shape
+    order = np.argsort(-lg, axis=1, kind="stable")
+    idx = np.full((T, k_max), -1)
+    for t in range(T):
+        n = 1
+        while n < k_max and p[t, order[t, n]] > delta:
+            n += 1
+        idx[t, :n] = order[t, :n]
+    return idx, p
+
+
+@pytest.mark.parametrize("E,k_max", [(4, 4), (8, 3), (16, 8), (32, 8)])
+def test_threshold_select_matches_definition(O, E, k_max):
+    lg = (rng.standard_normal((300, E)) * 1.5).astype(np.float32)
+    sel = O.threshold_select(lg, k_max)                              # default delta = 1/E
+    idx_ref, p = _threshold_reference(lg, k_max, 1.0 / E)
+    np.testing.assert_array_equal(sel["topk_idx"], idx_ref)
+    np.testing.assert_array_equal(sel["n_sel"], (idx_ref >= 0).sum(1))
+    g = sel["topk_gate"].astype(np.float64)
+    kept = idx_ref >= 0
+    assert np.all(np.abs(g.sum(1) - 1.0) <= 1e-6) and np.all(g[~kept] == 0)
+    pk = np.where(kept, np.take_along_axis(p, np.maximum(idx_ref, 0), 1), 0.0)
+    np.testing.assert_allclose(g, pk / pk.sum(1, keepdims=True), rtol=1e-6, atol=1e-7)
+
+
+def test_threshold_select_limits(O):
+    lg = rng.standard_normal((100, 6)).astype(np.float32)
+    # delta >= 1: nothing exceeds it, so only the largest is kept, with gate 1
+    one = O.threshold_select(lg, 4, 1.5)
+    np.testing.assert_array_equal(one["n_sel"], 1)
+    np.testing.assert_array_equal(one["topk_idx"][:, 0], np.argmax(lg, axis=1))
+    np.testing.assert_array_equal(one["topk_gate"][:, 0], 1.0)
+    # delta tiny and k_max = E: every expert kept, gates = the full softmax
+    every = O.threshold_select(lg, 6, 1e-30)
+    np.testing.assert_array_equal(every["topk_idx"], np.argsort(-lg, axis=1, kind="stable"))
+    np.testing.assert_allclose(np.sort(every["topk_gate"], axis=1),
+                               np.sort(softmax(lg.astype(np.float64), axis=1), axis=1), rtol=1e-6)
+
+
+def test_threshold_forward_reduces_to_topk_when_all_pass(O):
+    # delta tiny: every one of the k_max slots is used, so the layer is top-k_max gating
+    T, H, F, E, k = 48, 16, 24, 6, 2
+    x = PY.round_to_bf16(rng.standard_normal((T, H)))
+    wg = PY.round_to_bf16(rng.standard_normal((H, E)) / 4)
+    w1 = PY.round_to_bf16(rng.standard_normal((E, H, F)) / 4)
+    w3 = PY.round_to_bf16(rng.standard_normal((E, H, F)) / 4)
+    w2 = PY.round_to_bf16(rng.standard_normal((E, F, H)) / 5)
+    thr = O.moe_forward_threshold(x, wg, None, w1, w3, w2, k, 1e-30, 0.0, "swiglu", "bf16")
+    top = O.moe_forward(x, wg, None, w1, w3, w2, k, 0.0, "swiglu", "bf16")
+    np.testing.assert_array_equal(thr["topk_idx"], top["topk_idx"])
+    np.testing.assert_array_equal(thr["out"], top["out"])
+
+
+def test_permute_empty_slots(O):
+    idx = np.array([[1, -1, -1], [0, 2, -1], [2, 1, 0]], dtype=np.int32)
+    p = O.permute(idx, 3, None, empty_slots=True)
+    np.testing.assert_array_equal(p["counts"], [2, 2, 2])
+    np.testing.assert_array_equal(p["row_token"], [1, 2, 0, 2, 1, 2])
+    np.testing.assert_array_equal(p["row_map"], [[2, -1, -1], [0, 4, -1], [5, 3, 1]])
+    assert p["dropped"] == 0 and p["R"] == 6
+    with pytest.raises(O.IndexOutOfRange):
+        O.permute(idx, 3, None)                                     # -1 is an error otherwise
