@@ -250,6 +250,16 @@ moe_status moe_forward_threshold(const void* x, const void* w_gate, const float*
                                  int32_t* topk_idx_out, int32_t* n_selected_out,
                                  void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Self-test hook (no counterpart on the pages): applies, elementwise to fp32
+ * z[n] on the device, the activations the bf16 expert-GEMM epilogue uses
+ * before rounding h to bf16 — GELU z Phi(z) with Phi(z) = erfc(-z/sqrt 2)/2
+ * and erfc from the Numerical Recipes (2nd ed., section 6.2) Chebyshev fit
+ * (fractional error below 1.2e-7), and SiLU z / (1 + e^-z) with the hardware
+ * exponential and reciprocal — so tests can bound their error against exact
+ * values.  The fp32 path uses erfcf / expf.                                  */
+moe_status moe_selftest_epilogue_activations(const float* z, int n, float* gelu_out,
+                                             float* silu_out, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the status the kernels of the last
  * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */
 moe_status moe_get_device_status(void* ws, moe_stream_t stream);

@@ -72,7 +72,9 @@ bool ranks_before(float va, int ea, float vb, int eb) {
   return ea < eb;
 }
 
-double gelu(double z) { return 0.5 * z * (1.0 + std::erf(z / std::sqrt(2.0))); }
+// GELU(z) = z Phi(z) = 0.5 z (1 + erf(z / sqrt 2)), evaluated as 0.5 z erfc(-z / sqrt 2):
+// the same function without the cancellation of 1 + erf for z below about -5.
+double gelu(double z) { return 0.5 * z * std::erfc(-z / std::sqrt(2.0)); }
 double silu(double z) { return z / (1.0 + std::exp(-z)); }
 
 }  // namespace

@@ -43,7 +43,7 @@ import math
 from fractions import Fraction
 
 import numpy as np
-from scipy.special import erf as _erf
+from scipy.special import erfc as _erfc
 
 # --------------------------------------------------------------------------
 # Rounding to the storage dtype.
@@ -258,9 +258,11 @@ def permute(idx, E: int, cap=None, empty_slots: bool = False) -> dict:
 
 
 def gelu(z) -> np.ndarray:
-    """Exact GELU: 0.5 z (1 + erf(z / sqrt 2))."""
+    """Exact GELU: z * Phi(z) = 0.5 z (1 + erf(z / sqrt 2)), evaluated as
+    0.5 z erfc(-z / sqrt 2) (the same function; 1 + erf(x) = erfc(-x) avoids the
+    cancellation that loses all relative precision for z below about -5)."""
     z = np.asarray(z, dtype=np.float64)
-    return 0.5 * z * (1.0 + _erf(z / math.sqrt(2.0)))
+    return 0.5 * z * _erfc(-z / math.sqrt(2.0))
 
 
 def silu(z) -> np.ndarray:

@@ -56,6 +56,7 @@ _SIGS = {
     "moe_forward_threshold_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "moe_forward_threshold": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _i, _i, _p,
                                    _p, _p, _p, _sz, _p]),
+    "moe_selftest_epilogue_activations": (_i, [_p, _i, _p, _p, _p]),
     "moe_get_device_status": (_i, [_p, _p]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
@@ -407,6 +408,16 @@ def forward_threshold(x, w_gate, gate_bias, w1, w3, w2, k_max, delta=0.0, capaci
                                       _ptr(topk_idx_out), _ptr(n_selected_out), _ptr(ws),
                                       ws.numel(), _stream()), "moe_forward_threshold")
     return out, ws
+
+
+def epilogue_activations(z):
+    """(gelu, silu) of fp32 z as the bf16 GEMM epilogue computes them (self-test hook)."""
+    _need(z, "z", dtype=torch.float32)
+    z = z.contiguous()
+    g, s = torch.empty_like(z), torch.empty_like(z)
+    _check(_lib.moe_selftest_epilogue_activations(_ptr(z), z.numel(), _ptr(g), _ptr(s), _stream()),
+           "moe_selftest_epilogue_activations")
+    return g, s
 
 
 def device_status(ws) -> int:

@@ -351,6 +351,12 @@ MatmulWs matmul_ws(int T, int H, int I, int E, moe_dtype dt) {
 }
 }  // namespace
 
+moe_status moe_selftest_epilogue_activations(const float* z, int n, float* gelu_out,
+                                             float* silu_out, moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (!z || !gelu_out || !silu_out))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_epilogue_activations(z, n, gelu_out, silu_out, as_stream(stream)));
+}
+
 size_t moe_expert_matmul_workspace_bytes(int T, int H, int I, int E, moe_dtype dt) {
   if (T < 0 || H <= 0 || I <= 0 || E <= 0) return 0;
   return matmul_ws(T, H, I, E, dt).total;

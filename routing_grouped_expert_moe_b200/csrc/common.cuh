@@ -375,8 +375,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Exact-erf GELU and SiLU on fp32 values (the library's erff / expf).
+// GELU(z) = z Phi(z) = 0.5 z (1 + erf(z / sqrt 2)), as 0.5 z erfc(-z / sqrt 2):
+// the same function without the cancellation of 1 + erf for negative z.
 __device__ __forceinline__ float gelu_f(float z) {
-  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  return 0.5f * z * erfcf(-z * 0.70710678118654752f);
 }
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 

@@ -66,7 +66,58 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Registers written by an asynchronous tcgen05.ld are valid only after
+// tcgen05.wait::ld; this empty asm makes every later use depend on a point
+// after the wait, so the compiler cannot move a use above it.
+__device__ __forceinline__ void reg_fence32(float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+f"(v[i]));
+}
+
+// Activations of the bf16 tensor-core epilogue, whose results are rounded to
+// bf16 (relative spacing 2^-8), so a few fp32 ulps of error are invisible.
+//
+// GELU(z) = z Phi(z), Phi(z) = erfc(-z / sqrt 2) / 2.  erfc(x) for x >= 0 by the
+// Chebyshev fit of Press, Teukolsky, Vetterling & Flannery, Numerical Recipes
+// (2nd ed., section 6.2), fractional error below 1.2e-7 everywhere:
+//   erfc(x) = t exp(-x^2 + P(t)),  t = 1 / (1 + x/2),  P a degree-9 polynomial.
+// Then Phi(z) = 1 - erfc(|x|)/2 for z >= 0 and erfc(|x|)/2 for z < 0, so the
+// negative tail keeps its relative accuracy (1 + erf(x) would cancel).
+// Reciprocal by the special-function unit (about 1 ulp; denominators here are
+// at least 1, or infinite, giving 0).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ float erfc_nonneg(float ax) {
+  const float t = rcp_approx(fmaf(0.5f, ax, 1.0f));
+  float p = 0.17087277f;
+  p = fmaf(p, t, -0.82215223f);
+  p = fmaf(p, t, 1.48851587f);
+  p = fmaf(p, t, -1.13520398f);
+  p = fmaf(p, t, 0.27886807f);
+  p = fmaf(p, t, -0.18628806f);
+  p = fmaf(p, t, 0.09678418f);
+  p = fmaf(p, t, 0.37409196f);
+  p = fmaf(p, t, 1.00002368f);
+  p = fmaf(p, t, -1.26551223f);
+  return t * __expf(fmaf(-ax, ax, p));
+}
+
+__device__ __forceinline__ float gelu_epi(float z) {
+  const float e = erfc_nonneg(fabsf(z) * 0.70710678118654752f);
+  return z * (z >= 0.f ? fmaf(-0.5f, e, 1.0f) : 0.5f * e);
+}
+
+// SiLU with the hardware exponential and reciprocal: z / (1 + e^-z).
+__device__ __forceinline__ float silu_epi(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 
 // Activation of one thread's 32 accumulator columns, packed to bf16 pairs.
 template <int MODE>
@@ -75,28 +126,36 @@ __device__ __forceinline__ void epilogue_pack(const float (&v)[32], const float 
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float a0 = v[2 * i], a1 = v[2 * i + 1];
-    if (MODE == 0) { a0 = gelu_f(a0); a1 = gelu_f(a1); }
-    if (MODE == 1) { a0 = silu_f(a0) * u[2 * i]; a1 = silu_f(a1) * u[2 * i + 1]; }
+    if (MODE == 0) { a0 = gelu_epi(a0); a1 = gelu_epi(a1); }
+    if (MODE == 1) { a0 = silu_epi(a0) * u[2 * i]; a1 = silu_epi(a1) * u[2 * i + 1]; }
     p[i] = pack_bf16x2(a0, a1);
   }
 }
 
 // Writes one warp's 32 rows x 32 columns of output.  When all 32 rows belong
-// to the tile's expert, the rows go through the warp's 2 KB staging box in
+// to the tile's expert, the rows go through one of the warp's staging boxes in
 // shared memory and one TMA bulk store (columns past N are clipped by the
 // tensor map); otherwise (the ragged end of an expert, whose following rows
-// belong to the next expert) each thread stores its own row, masked.
+// belong to the next expert) each thread stores its own row, masked.  With
+// two boxes used in turn, a box is rewritten only after the store issued from
+// it two chunks earlier has read it (wait_group.read 1), unless the last
+// committed store came from the same box (then wait for all).
 template <int MODE>
 __device__ __forceinline__ void epilogue_chunk(const float (&v)[32], const float (&u)[32],
-                                               const CUtensorMap* tmO, uint8_t* stg, int lane,
-                                               bool box_full, int out_row0, int col0, int N,
+                                               const CUtensorMap* tmO, uint8_t* stg_base, int box,
+                                               int& last_box, int lane, bool box_full,
+                                               int out_row0, int col0, int N,
                                                __nv_bfloat16* orow, bool row_ok) {
   uint32_t p[16];
   epilogue_pack<MODE>(v, u, p);
   const int cols_left = N - col0;
   if (cols_left <= 0) return;
   if (box_full) {
-    if (lane == 0) bulk_wait_read0();  // the previous store has read the box
+    uint8_t* stg = stg_base + box * G_STG_BYTES;
+    if (lane == 0) {
+      if (box == last_box) bulk_wait_read0();
+      else bulk_wait_read1();
+    }
     __syncwarp();
     // row `lane` = 64 bytes; 16-byte pieces in rotated order spread the banks
     const uint4 q0 = make_uint4(p[0], p[1], p[2], p[3]);
@@ -115,11 +174,61 @@ __device__ __forceinline__ void epilogue_chunk(const float (&v)[32], const float
       tma_store_2d(tmO, stg, col0, out_row0);
       bulk_commit();
     }
+    last_box = box;
   } else if (row_ok) {
     uint4* d = reinterpret_cast<uint4*>(orow);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       if (8 * j < cols_left) d[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+  }
+}
+
+// One epilogue warp's share of a finished accumulator tile (its 32 TMEM lanes,
+// one half of the columns): TMEM -> registers -> activation -> bf16 -> global.
+// Modes 0 and 2 (four 32-column chunks) load the next chunk from TMEM before
+// working on the current one, so the load latency hides behind the
+// activation; mode 1 reads the W1 and W3 halves of two chunks.  NBOX staging
+// boxes (1 or 2) are used in turn.
+template <int MODE, int NBOX>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int half, const CUtensorMap* tmO,
+                                              uint8_t* stg, int& last_box, int lane,
+                                              bool box_full, bool row_ok, int out_row0, int n0,
+                                              int N, __nv_bfloat16* orow) {
+  constexpr int B1 = NBOX > 1 ? 1 : 0;
+  if (MODE == 1) {
+#pragma unroll 1
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
+      float g[32], u[32];
+      tmem_ld32(t_row + c * 32, g);
+      tmem_ld32(t_row + 128 + c * 32, u);
+      tmem_ld_wait();
+      reg_fence32(g);
+      reg_fence32(u);
+      epilogue_chunk<1>(g, u, tmO, stg, (c & 1) ? B1 : 0, last_box, lane, box_full, out_row0,
+                        n0 + c * 32, N, row_ok ? orow + c * 32 : nullptr, row_ok);
+    }
+  } else {
+    const int c0 = 4 * half;
+    float va[32], vb[32];
+    tmem_ld32(t_row + c0 * 32, va);
+    tmem_ld_wait();
+    reg_fence32(va);
+#pragma unroll 1
+    for (int i = 0; i < 4; i += 2) {
+      const int c = c0 + i;
+      tmem_ld32(t_row + (c + 1) * 32, vb);
+      epilogue_chunk<MODE>(va, va, tmO, stg, 0, last_box, lane, box_full, out_row0, n0 + c * 32,
+                           N, row_ok ? orow + c * 32 : nullptr, row_ok);
+      tmem_ld_wait();
+      reg_fence32(vb);
+      if (i + 2 < 4) tmem_ld32(t_row + (c + 2) * 32, va);
+      epilogue_chunk<MODE>(vb, vb, tmO, stg, B1, last_box, lane, box_full, out_row0,
+                           n0 + (c + 1) * 32, N, row_ok ? orow + (c + 1) * 32 : nullptr, row_ok);
+      if (i + 2 < 4) {
+        tmem_ld_wait();
+        reg_fence32(va);
+      }
+    }
   }
 }
 

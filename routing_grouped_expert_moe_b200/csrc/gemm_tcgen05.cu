@@ -225,7 +225,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
-    uint8_t* stg = smem + G_STAGES * G_STAGE_BYTES + (warp - 2) * G_STG_BYTES;  // this warp's staging box
+    uint8_t* stg = smem + G_STAGES * G_STAGE_BYTES + (warp - 2) * 1 * G_STG_BYTES;  // this warp's staging boxes
+    int last_box = -1;  // box of the last committed bulk store
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -241,26 +242,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
-      if (MODE == 1) {
-#pragma unroll 1
-        for (int c = 2 * half; c < 2 * half + 2; ++c) {
-          float g[32], u[32];
-          tmem_ld32(t_row + c * 32, g);
-          tmem_ld32(t_row + 128 + c * 32, u);
-          tmem_ld_wait();
-          epilogue_chunk<1>(g, u, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32, args.N,
-                            row_ok ? orow + c * 32 : nullptr, row_ok);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 4 * half; c < 4 * half + 4; ++c) {
-          float v[32];
-          tmem_ld32(t_row + c * 32, v);
-          tmem_ld_wait();
-          epilogue_chunk<MODE>(v, v, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32,
-                               args.N, row_ok ? orow + c * 32 : nullptr, row_ok);
-        }
-      }
+      epilogue_tile<MODE, 1>(t_row, half, &tmO, stg, last_box, lane, box_full, row_ok,
+                                 ti.m0 + q * 32, ti.n0, args.N, orow);
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -273,6 +256,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, G_TMEM_COLS);
   }
+}
+
+// The activations the bf16 epilogue applies, elementwise (self-test hook).
+__global__ void k_epilogue_activations(const float* __restrict__ z, int n, float* __restrict__ gelu,
+                                       float* __restrict__ silu) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    gelu[i] = gelu_epi(z[i]);
+    silu[i] = silu_epi(z[i]);
+  }
+}
+
+cudaError_t launch_epilogue_activations(const float* z, int n, float* gelu, float* silu,
+                                        cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  k_epilogue_activations<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s>>>(z, n, gelu,
+                                                                                      silu);
+  return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------------------

@@ -4,10 +4,10 @@
 // (lshu.cn torch_npu fused-operator article §3-§4: per-expert x W1 [, x W3],
 // activation, and the down-projection), but two CTAs of a cluster share one
 // 256 x 256 x 64 MMA: each CTA stages its own 128 A rows and one half of the
-// 256 B columns, so every SM moves 32 KB per k-block instead of 48 KB and the
-// TMA ring deepens from 4 to 6 stages.  The pair's rows are two consecutive
-// 128-row m-tiles of the same expert (an odd last m-tile leaves the second
-// CTA's rows empty: computed, never stored).
+// 256 B columns, so every SM moves 32 KB per k-block instead of 48 KB; the
+// ring has 5 stages and each epilogue warp two staging boxes.  The pair's rows
+// are two consecutive 128-row m-tiles of the same expert (an odd last m-tile
+// leaves the second CTA's rows empty: computed, never stored).
 //
 // Roles per CTA (320 threads): warp 0 TMA producer (both CTAs; completion is
 // counted on the first CTA's full barrier), warp 1 MMA issuer (first CTA only)
@@ -19,11 +19,11 @@
 
 namespace moe {
 
-constexpr int P_STAGES = 6;
+constexpr int P_STAGES = 5;
 constexpr int P_A_BYTES = G_BM * G_BK * 2;            // 16 KB: this CTA's 128 rows
 constexpr int P_B_BYTES = (G_ACC_N / 2) * G_BK * 2;   // 16 KB: half of the 256 columns
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;  // 32 KB
-constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + G_EPI_WARPS * G_STG_BYTES + 1024;
+constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + G_EPI_WARPS * 2 * G_STG_BYTES + 1024;
 
 struct PairTile {
   int e, n0, m0, rows, seg_start;
@@ -243,7 +243,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
-    uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES + (warp - 2) * G_STG_BYTES;  // this warp's staging box
+    uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES + (warp - 2) * 2 * G_STG_BYTES;  // this warp's staging boxes
+    int last_box = -1;  // box of the last committed bulk store
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -260,26 +261,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
-      if (MODE == 1) {
-#pragma unroll 1
-        for (int c = 2 * half; c < 2 * half + 2; ++c) {
-          float g[32], u[32];
-          tmem_ld32(t_row + c * 32, g);
-          tmem_ld32(t_row + 128 + c * 32, u);
-          tmem_ld_wait();
-          epilogue_chunk<1>(g, u, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32, args.N,
-                            row_ok ? orow + c * 32 : nullptr, row_ok);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 4 * half; c < 4 * half + 4; ++c) {
-          float v[32];
-          tmem_ld32(t_row + c * 32, v);
-          tmem_ld_wait();
-          epilogue_chunk<MODE>(v, v, &tmO, stg, lane, box_full, ti.m0 + q * 32, ti.n0 + c * 32,
-                               args.N, row_ok ? orow + c * 32 : nullptr, row_ok);
-        }
-      }
+      epilogue_tile<MODE, 2>(t_row, half, &tmO, stg, last_box, lane, box_full, row_ok,
+                                 ti.m0 + q * 32, ti.n0, args.N, orow);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty_bar[acc]), 0));

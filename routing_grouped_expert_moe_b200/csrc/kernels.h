@@ -89,6 +89,9 @@ cudaError_t launch_gemm_tc_pair(int mode, bool gather, const CUtensorMap& ma,
                                 const CUtensorMap& mb1, const CUtensorMap& mb3,
                                 const CUtensorMap& mo, const GemmArgs& g, int num_sms,
                                 cudaStream_t s);
+// The bf16 epilogue's activations applied elementwise (self-test hook).
+cudaError_t launch_epilogue_activations(const float* z, int n, float* gelu, float* silu,
+                                        cudaStream_t s);
 // fp32 CUDA-core path (no TF32).
 cudaError_t launch_gemm_simt(int mode, const void* a_src, const void* b1, const void* b3,
                              const GemmArgs& g, int num_sms, cudaStream_t s);
