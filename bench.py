@@ -473,7 +473,7 @@ def main(argv=None):
     total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(T, world, args.steps, total_ms)
-    gpu_launches = 7 * args.steps
+    gpu_launches = 6 * args.steps   # clear-status, route, scatter (+scan), GEMM-1, GEMM-2, combine
 
     # ---- per-stage times of the same fused path (events at stage boundaries)
     n_stage = min(args.steps, 50)

@@ -3,6 +3,7 @@
 // point allocates device memory or synchronises the stream (except
 // moe_get_device_status, whose job is to synchronise).
 #include <climits>
+#include <cstdlib>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -11,6 +12,13 @@
 #include "moe_b200.h"
 
 using namespace moe;
+
+namespace moe {
+bool pdl_enabled() {
+  const char* e = getenv("MOE_PDL");
+  return !(e && e[0] == '0');
+}
+}  // namespace moe
 
 namespace {
 
@@ -233,7 +241,6 @@ moe_status moe_permute(const void* x, const int32_t* token_expert_idx, int T, in
     return cuda_status(cudaMemsetAsync(expert_offsets, 0, (E + 1) * 4, s));
   }
   if (launch_hist(p, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_scan(p, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(launch_scatter(p, s));
 }
 
@@ -397,7 +404,6 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
   p.x = x; p.x_perm = x_perm; p.H = H; p.elem_bytes = elem_bytes(dt);
   p.status = status;
   if (launch_hist(p, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_scan(p, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_scatter(p, s) != cudaSuccess) return MOE_ERR_CUDA;
   // per-expert matmul of the expert-major rows: y = x_perm W[e]
   GemmArgs g{};
@@ -502,7 +508,9 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
     if (launch_hist(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (mark(1) != cudaSuccess) return MOE_ERR_CUDA;
-  // 2. scan + scatter over the router's (or the histogram's) token tiles
+  // 2. scatter (the per-expert scan over tiles runs in its prologue) over the
+  // router's (or the histogram's) token tiles; the "scan" stage events stay
+  // for the callers that time stages, with nothing between them
   // enough scatter CTAs to keep the x_perm row copies near HBM bandwidth
   pa.split = 1;
   if (x_perm)
@@ -510,7 +518,6 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   pa.cap = capacity_of(capacity_factor, T, top_k, E);
   pa.counts = counts; pa.offsets = offsets; pa.row_token = row_token; pa.row_map = row_map;
   pa.x = x; pa.x_perm = x_perm; pa.H = H; pa.elem_bytes = elem_bytes(dt);
-  if (launch_scan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (mark(2) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_scatter(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (mark(3) != cudaSuccess) return MOE_ERR_CUDA;

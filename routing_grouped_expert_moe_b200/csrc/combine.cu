@@ -21,6 +21,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kCombineThreads)
     k_combine(const uint8_t* __restrict__ y, const float* __restrict__ gate,
               const int32_t* __restrict__ row_map, int T, int H, int k, uint8_t* __restrict__ out) {
+  pdl_wait_and_trigger();
   constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
   constexpr int EB = BF16 ? 2 : 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -84,12 +85,12 @@ cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   if (dt_bf16)
-    k_combine<true><<<grid, kCombineThreads, 0, s>>>(static_cast<const uint8_t*>(y), gate, row_map,
-                                                     T, H, k, static_cast<uint8_t*>(out));
-  else
-    k_combine<false><<<grid, kCombineThreads, 0, s>>>(static_cast<const uint8_t*>(y), gate,
-                                                      row_map, T, H, k, static_cast<uint8_t*>(out));
-  return cudaGetLastError();
+    return launch_kernel(k_combine<true>, dim3(grid), dim3(kCombineThreads), 0, s, 1,
+                         static_cast<const uint8_t*>(y), gate, row_map, T, H, k,
+                         static_cast<uint8_t*>(out));
+  return launch_kernel(k_combine<false>, dim3(grid), dim3(kCombineThreads), 0, s, 1,
+                       static_cast<const uint8_t*>(y), gate, row_map, T, H, k,
+                       static_cast<uint8_t*>(out));
 }
 
 }  // namespace moe

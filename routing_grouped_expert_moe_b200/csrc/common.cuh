@@ -25,6 +25,15 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);  // the first error wins
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on has
+// completed (no-op without such a dependency), then let the next grid in the
+// stream be scheduled (its own wait keeps it from reading this grid's output
+// before this grid completes).
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(S_THREADS)
   __shared__ float Bs[S_BK][S_BN];
   __shared__ float B3s[MODE == 1 ? S_BK : 1][MODE == 1 ? S_BN : 1];
   __shared__ int s_prefix[kMaxE + 1], s_start[kMaxE], s_rows[kMaxE], s_mt[kMaxE];
+  pdl_wait_and_trigger();
   __shared__ int s_arow[S_BM];
   const int E = args.E, N = args.N, K = args.K;
   const int ntn = (N + S_BN - 1) / S_BN;
@@ -122,20 +123,21 @@ cudaError_t launch_gemm_simt(int mode, const void* a_src, const void* b1, const 
   const float* W3 = static_cast<const float*>(b3);
   const bool gather = g.row_token != nullptr;
   const int grid = num_sms * 2;
+  const dim3 gd(grid), bd(S_THREADS);
   switch (mode * 2 + (gather ? 1 : 0)) {
-    case 0: k_gemm_simt<0, false><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
-    case 1: k_gemm_simt<0, true><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
-    case 2: k_gemm_simt<1, false><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
-    case 3: k_gemm_simt<1, true><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
-    case 4: k_gemm_simt<2, false><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
-    case 5: k_gemm_simt<2, true><<<grid, S_THREADS, 0, s>>>(A, W1, W3, g); break;
+    case 0: return launch_kernel(k_gemm_simt<0, false>, gd, bd, 0, s, 1, A, W1, W3, g);
+    case 1: return launch_kernel(k_gemm_simt<0, true>, gd, bd, 0, s, 1, A, W1, W3, g);
+    case 2: return launch_kernel(k_gemm_simt<1, false>, gd, bd, 0, s, 1, A, W1, W3, g);
+    case 3: return launch_kernel(k_gemm_simt<1, true>, gd, bd, 0, s, 1, A, W1, W3, g);
+    case 4: return launch_kernel(k_gemm_simt<2, false>, gd, bd, 0, s, 1, A, W1, W3, g);
+    case 5: return launch_kernel(k_gemm_simt<2, true>, gd, bd, 0, s, 1, A, W1, W3, g);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 // Identity experts: out[r] = A[row_token[r]] (gather) or A[r], for r < offsets[E].
 __global__ void k_copy_rows(const uint8_t* __restrict__ A, const GemmArgs g, int row_bytes) {
+  pdl_wait_and_trigger();
   const int R = min(g.offsets[g.E], g.R_max);
   const int vecs = row_bytes / 16;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -150,8 +152,8 @@ __global__ void k_copy_rows(const uint8_t* __restrict__ A, const GemmArgs g, int
 }
 
 cudaError_t launch_copy_rows(const void* a_src, const GemmArgs& g, int elem_bytes, cudaStream_t s) {
-  k_copy_rows<<<1184, 256, 0, s>>>(static_cast<const uint8_t*>(a_src), g, g.N * elem_bytes);
-  return cudaGetLastError();
+  return launch_kernel(k_copy_rows, dim3(1184), dim3(256), 0, s, 1,
+                       static_cast<const uint8_t*>(a_src), g, g.N * elem_bytes);
 }
 
 }  // namespace moe

@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     abort_s = 0;
     fence_mbar_init();
   }
+  pdl_wait_and_trigger();  // expert offsets and A rows come from the previous kernel
   if (warp == 0) {
     // Tile schedule from the expert segments: tiles(e) = ceil(rows_e/128) * n_tiles.
     int carry = 0;
@@ -261,6 +262,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 // The activations the bf16 epilogue applies, elementwise (self-test hook).
 __global__ void k_epilogue_activations(const float* __restrict__ z, int n, float* __restrict__ gelu,
                                        float* __restrict__ silu) {
+  pdl_wait_and_trigger();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     gelu[i] = gelu_epi(z[i]);
     silu[i] = silu_epi(z[i]);
@@ -270,9 +272,8 @@ __global__ void k_epilogue_activations(const float* __restrict__ z, int n, float
 cudaError_t launch_epilogue_activations(const float* z, int n, float* gelu, float* silu,
                                         cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  k_epilogue_activations<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, s>>>(z, n, gelu,
-                                                                                      silu);
-  return cudaGetLastError();
+  return launch_kernel(k_epilogue_activations, dim3((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024),
+                       dim3(256), 0, s, 1, z, n, gelu, silu);
 }
 
 // ----------------------------------------------------------------------------
@@ -284,8 +285,7 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const 
   auto kern = k_gemm_tc<MODE, GATHER>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
   if (err != cudaSuccess) return err;
-  kern<<<num_sms, G_THREADS, G_SMEM, s>>>(a, b1, b3, o, g);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(num_sms), dim3(G_THREADS), G_SMEM, s, 1, a, b1, b3, o, g);
 }
 
 // Kernel variant: one CTA per 128-row tile, or CTA pairs sharing 256-row

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     abort_s = 0;
     fence_mbar_init();
   }
+  pdl_wait_and_trigger();  // expert offsets and A rows come from the previous kernel
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < E; base += 32) {
@@ -286,19 +287,8 @@ static cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b1, cons
   auto kern = k_gemm_tc_pair<MODE, GATHER>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((num_sms / 2) * 2, 1, 1);
-  cfg.blockDim = dim3(G_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = P_SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, b1, b3, o, g);
+  return launch_kernel(kern, dim3((num_sms / 2) * 2), dim3(G_THREADS), P_SMEM, s, 2, a, b1, b3, o,
+                       g);
 }
 
 cudaError_t launch_gemm_tc_pair(int mode, bool gather, const CUtensorMap& ma,

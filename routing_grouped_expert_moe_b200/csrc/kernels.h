@@ -10,6 +10,41 @@ namespace moe {
 constexpr int kMaxE = 256;
 constexpr int kMaxTopK = 8;
 
+// ---------------------------------------------------------------- launches
+// Programmatic dependent launch: with it on, a kernel's CTAs may be scheduled
+// while its predecessor in the stream is finishing, and run their prologue;
+// every kernel of this library executes griddepcontrol.wait (pdl_wait) before
+// it touches global memory, which returns once the predecessor grid has
+// completed and its writes are visible.  MOE_PDL=0 turns the attribute off.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ---------------------------------------------------------------- router
 struct RouteArgs {
   const void* x;        // [T,H] bf16 or fp32
@@ -47,7 +82,7 @@ struct PermuteArgs {
   int tiles;
   int split;            // CTAs per tile in the scatter (share the x_perm row copies)
   int cap;              // per-expert capacity (INT32_MAX when unlimited)
-  int* tile_counts;     // [tiles,E] histogram in, tile bases out (in place)
+  int* tile_counts;     // [tiles,E] per-tile expert histogram (read by the scatter)
   int32_t* counts;      // [E]   pre-drop counts
   int32_t* offsets;     // [E+1] post-drop exclusive prefix
   int32_t* row_token;   // [T*k]
@@ -61,7 +96,6 @@ struct PermuteArgs {
 
 constexpr int kPermuteBT = 128;
 cudaError_t launch_hist(const PermuteArgs& a, cudaStream_t s);
-cudaError_t launch_scan(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- grouped GEMM

@@ -125,6 +125,5 @@ extern "C" moe_status moe_permute_noalloc(const void* x, const int32_t* token_ex
   p.elem_bytes = eb;
   p.status = status;
   if (launch_hist(p, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_scan(p, s) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_scatter(p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

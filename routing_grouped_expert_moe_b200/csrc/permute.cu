@@ -9,10 +9,11 @@
 // CSR storage of the sparse assignment).
 //
 // Pairs are ordered by a = t*k + s.  The tokens are cut into tiles of BT; the
-// histogram gives per-tile counts, one CTA scans them per expert (tile bases,
-// pre-drop counts, capacity clamp, offsets), and the scatter recomputes each
-// pair's rank inside its tile with warp match/popc, so rank = tile base + rank
-// in tile is the pair's arrival order among all pairs of that expert.
+// histogram gives per-tile counts; each scatter CTA scans them per expert for
+// its own tile base (plus pre-drop counts, capacity clamp and offsets) and
+// recomputes each pair's rank inside its tile with warp match/popc, so rank =
+// tile base + rank in tile is the pair's arrival order among all pairs of
+// that expert.
 #include <climits>
 
 #include "common.cuh"
@@ -27,6 +28,7 @@ constexpr int kPermThreads = 256;
 // empty_slots, id -1 is an unused slot and is skipped silently.
 __global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
   __shared__ int cnt_s[kMaxE];
+  pdl_wait_and_trigger();
   const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < a.E; i += kPermThreads) cnt_s[i] = 0;
   __syncthreads();
@@ -50,80 +52,86 @@ __global__ void __launch_bounds__(kPermThreads) k_hist(PermuteArgs a) {
     a.tile_counts[static_cast<size_t>(blockIdx.x) * a.E + i] = cnt_s[i];
 }
 
-// One CTA: per-expert exclusive scan over tiles (written back in place as
-// tile bases), pre-drop counts, kept = min(count, C), offsets = scan(kept).
-// Thread (p, e) owns a contiguous run of tiles of expert e: it sums the run,
-// one block scan over p gives each run's base, and a second pass writes the
-// bases; consecutive threads read consecutive experts of a tile (coalesced).
-constexpr int kScanThreads = 1024;
-
-__global__ void __launch_bounds__(kScanThreads) k_scan(PermuteArgs a) {
-  __shared__ int buf[kScanThreads];
-  __shared__ int total[kMaxE];
-  int Ep = 1;
-  while (Ep < a.E) Ep <<= 1;
-  const int P = kScanThreads / Ep;  // runs per expert
-  const int e = threadIdx.x % Ep, p = threadIdx.x / Ep;
-  const int run = (a.tiles + P - 1) / P;
-  const int j0 = p * run, j1 = min(a.tiles, j0 + run);
-  int sum = 0;
-  if (e < a.E)
-    for (int j = j0; j < j1; ++j) sum += a.tile_counts[static_cast<size_t>(j) * a.E + e];
-  buf[threadIdx.x] = sum;
-  __syncthreads();
-  for (int off = 1; off < P; off <<= 1) {
-    const int u = (p >= off) ? buf[threadIdx.x - off * Ep] : 0;
-    __syncthreads();
-    buf[threadIdx.x] += u;
-    __syncthreads();
-  }
-  if (e < a.E) {
-    int base = buf[threadIdx.x] - sum;  // exclusive prefix of this run
-    for (int j = j0; j < j1; ++j) {
-      const size_t i = static_cast<size_t>(j) * a.E + e;
-      const int v = a.tile_counts[i];
-      a.tile_counts[i] = base;
-      base += v;
-    }
-    if (p == P - 1) total[e] = buf[threadIdx.x];
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    int acc = 0;
-    for (int b = 0; b < a.E; b += 32) {
-      const int ee = b + threadIdx.x;
-      int kept = 0;
-      if (ee < a.E) {
-        a.counts[ee] = total[ee];
-        kept = min(total[ee], a.cap);
-      }
-      int incl = kept;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, off);
-        if (threadIdx.x >= off) incl += u;
-      }
-      if (ee < a.E) a.offsets[ee] = acc + incl - kept;
-      acc += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (threadIdx.x == 0) a.offsets[a.E] = acc;
-  }
-}
-
-// Stable scatter.  CTA j handles pairs [j*BT*k, min(T,(j+1)*BT)*k) in rounds
-// of 256; inside a round a pair's rank among same-expert pairs comes from
-// __match_any_sync (rank in warp) plus an exclusive scan over warps.
+// Stable scatter with the scan folded in.  CTA j handles pairs
+// [j*BT*k, min(T,(j+1)*BT)*k) in rounds of 256.
+//
+// Prologue (every CTA, from the per-tile histogram): for each expert, the
+// pairs routed to it in tiles before j (this tile's base), the total over all
+// tiles (the pre-drop count), kept = min(count, C) and offsets = exclusive
+// scan of kept over experts.  Thread (p, e) sums a contiguous run of tiles of
+// expert e (consecutive threads read consecutive experts of a tile), then the
+// runs are added in order; CTA 0 also writes counts and offsets.  Integer
+// sums: every CTA gets the same values.
+//
+// Main loop: inside a round a pair's rank among same-expert pairs comes from
+// __match_any_sync (rank in warp) plus an exclusive scan over warps, so
+// rank = tile base + rank in tile is the pair's arrival order among all pairs
+// of its expert.
 constexpr int kScatterMaxPairs = 128 * kMaxTopK;
 
 __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
   __shared__ int wcnt[kPermThreads / 32][kMaxE];
   __shared__ int running[kMaxE];
   __shared__ int rows_s[kScatterMaxPairs];
+  __shared__ int part_all[kPermThreads], part_before[kPermThreads];
+  __shared__ int base_s[kMaxE], total_s[kMaxE], off_s[kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.split > 0 ? a.split : 1;
   const int j = blockIdx.x / split, part = blockIdx.x % split;  // tile, share of its copies
   const int a0 = j * a.BT * a.k;
   const int a1 = min(a.T, (j + 1) * a.BT) * a.k;
+  pdl_wait_and_trigger();
+
+  {  // ---- scan prologue
+    int Ep = 1;
+    while (Ep < a.E) Ep <<= 1;
+    const int P = kPermThreads / Ep;  // runs per expert (E <= 256)
+    const int e = threadIdx.x % Ep, p = threadIdx.x / Ep;
+    const int run = (a.tiles + P - 1) / P;
+    const int j0 = p * run, j1 = min(a.tiles, j0 + run);
+    int s_all = 0, s_before = 0;
+    if (e < a.E)
+      for (int jj = j0; jj < j1; ++jj) {
+        const int v = a.tile_counts[static_cast<size_t>(jj) * a.E + e];
+        s_all += v;
+        if (jj < j) s_before += v;
+      }
+    part_all[threadIdx.x] = s_all;
+    part_before[threadIdx.x] = s_before;
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < a.E; ee += kPermThreads) {
+      int tot = 0, bef = 0;
+      for (int q = 0; q < P; ++q) {
+        tot += part_all[q * Ep + ee];
+        bef += part_before[q * Ep + ee];
+      }
+      total_s[ee] = tot;
+      base_s[ee] = bef;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int acc = 0;
+      for (int b = 0; b < a.E; b += 32) {
+        const int ee = b + lane;
+        const int kept = ee < a.E ? min(total_s[ee], a.cap) : 0;
+        int incl = kept;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += u;
+        }
+        if (ee < a.E) {
+          off_s[ee] = acc + incl - kept;
+          if (blockIdx.x == 0) {
+            a.counts[ee] = total_s[ee];
+            a.offsets[ee] = acc + incl - kept;
+          }
+        }
+        acc += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (blockIdx.x == 0 && lane == 0) a.offsets[a.E] = acc;
+    }
+  }
   for (int i = threadIdx.x; i < a.E; i += kPermThreads) running[i] = 0;
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int base = a0; base < a1; base += kPermThreads) {
@@ -154,9 +162,9 @@ __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
     if (i < a1) {
       int row = -1;
       if (e >= 0) {
-        const int rank = a.tile_counts[static_cast<size_t>(j) * a.E + e] + wcnt[warp][e] + rank_w;
+        const int rank = base_s[e] + wcnt[warp][e] + rank_w;
         if (rank < a.cap) {
-          row = a.offsets[e] + rank;
+          row = off_s[e] + rank;
           if (part == 0) a.row_token[row] = i / a.k;
         }
       }
@@ -185,30 +193,25 @@ __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
 }
 
 cudaError_t launch_hist(const PermuteArgs& a, cudaStream_t s) {
-  k_hist<<<a.tiles, kPermThreads, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scan(const PermuteArgs& a, cudaStream_t s) {
-  k_scan<<<1, kScanThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(k_hist, dim3(a.tiles), dim3(kPermThreads), 0, s, 1, a);
 }
 
 cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s) {
   if (a.BT * a.k > kScatterMaxPairs) return cudaErrorInvalidValue;
-  k_scatter<<<a.tiles * (a.split > 0 ? a.split : 1), kPermThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(k_scatter, dim3(a.tiles * (a.split > 0 ? a.split : 1)), dim3(kPermThreads),
+                       0, s, 1, a);
 }
 
 __global__ void k_clear_status(int* status, int* counters, int n) {
+  pdl_wait_and_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
     counters[i] = 0;
 }
 
 cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters, int n) {
-  k_clear_status<<<1, 256, 0, s>>>(status, counters, counters ? n : 0);
-  return cudaGetLastError();
+  return launch_kernel(k_clear_status, dim3(1), dim3(256), 0, s, 1, status, counters,
+                       counters ? n : 0);
 }
 
 }  // namespace moe

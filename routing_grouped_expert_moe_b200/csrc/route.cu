@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_simt(RouteArgs a) {
   int* cnt_s = sel_s + kSimtBT * 8;                                 // [256]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int token0 = blockIdx.x * kSimtBT;
+  pdl_wait_and_trigger();
   const Tin* x = static_cast<const Tin*>(a.x);
   const Tin* wg = static_cast<const Tin*>(a.wg);
   for (int lt = warp; lt < kSimtBT; lt += kRouteThreads / 32) {
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_from_logits(RouteArgs a
   int* sel_s = reinterpret_cast<int*>(lg + kSimtBT * a.E);
   int* cnt_s = sel_s + kSimtBT * 8;
   const int token0 = blockIdx.x * kSimtBT;
+  pdl_wait_and_trigger();
   for (int i = threadIdx.x; i < kSimtBT * a.E; i += kRouteThreads) {
     const int t = token0 + i / a.E;
     lg[i] = t < a.T ? logits[static_cast<size_t>(token0) * a.E + i] : 0.f;
@@ -201,17 +203,15 @@ cudaError_t launch_route(const RouteArgs& a, const RoutePlan& p, cudaStream_t s)
   if (p.kind == 2) return launch_route_tc(a, p, s);
   const size_t smem = (kSimtBT * a.E + kSimtBT * 8 + 256) * 4;
   if (a.dt_bf16)
-    k_route_simt<__nv_bfloat16><<<p.tiles, kRouteThreads, smem, s>>>(a);
-  else
-    k_route_simt<float><<<p.tiles, kRouteThreads, smem, s>>>(a);
-  return cudaGetLastError();
+    return launch_kernel(k_route_simt<__nv_bfloat16>, dim3(p.tiles), dim3(kRouteThreads), smem, s,
+                         1, a);
+  return launch_kernel(k_route_simt<float>, dim3(p.tiles), dim3(kRouteThreads), smem, s, 1, a);
 }
 
 cudaError_t launch_route_from_logits(const RouteArgs& a, const float* logits, cudaStream_t s) {
   const int tiles = (a.T + kSimtBT - 1) / kSimtBT;
   const size_t smem = (kSimtBT * a.E + kSimtBT * 8 + 256) * 4;
-  k_route_from_logits<<<tiles, kRouteThreads, smem, s>>>(a, logits);
-  return cudaGetLastError();
+  return launch_kernel(k_route_from_logits, dim3(tiles), dim3(kRouteThreads), smem, s, 1, a, logits);
 }
 
 }  // namespace moe

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(R_THREADS)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait_and_trigger();
   const uint32_t tmem_base = tmem_base_s;
   volatile int* abort_flag = &abort_s;
 
@@ -323,8 +324,7 @@ static cudaError_t launch_route_tc_nk(const CUtensorMap& mx, const CUtensorMap& 
   auto kern = k_route_tc<NPAD, K>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
-  kern<<<dim3(tiles, S, 1), R_THREADS, C::SMEM, s>>>(mx, mw, a, S);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(tiles, S, 1), dim3(R_THREADS), C::SMEM, s, 1, mx, mw, a, S);
 }
 
 template <int NPAD>

@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(kThrThreads)
     k_route_threshold(const float* __restrict__ logits, int T, int E, int k_max, float delta,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
                       int32_t* __restrict__ n_sel) {
+  pdl_wait_and_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kThrWarps + warp;
   if (t >= T) return;
@@ -91,6 +92,7 @@ constexpr int kScanT = 1024;
 __global__ void __launch_bounds__(kScanT)
     k_token_offsets(const int32_t* __restrict__ n, int T, int32_t* __restrict__ out) {
   __shared__ int part[kScanT];
+  pdl_wait_and_trigger();
   const int per = (T + kScanT - 1) / kScanT;
   const int b = threadIdx.x * per, e = min(T, b + per);
   int s = 0;
@@ -115,13 +117,13 @@ cudaError_t launch_route_threshold(const float* logits, int T, int E, int k_max,
                                    int32_t* idx, float* gate, int32_t* n_sel,
                                    int32_t* token_offsets, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  k_route_threshold<<<(T + kThrWarps - 1) / kThrWarps, kThrThreads, 0, s>>>(logits, T, E, k_max,
-                                                                            delta, idx, gate, n_sel);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_kernel(k_route_threshold, dim3((T + kThrWarps - 1) / kThrWarps),
+                                  dim3(kThrThreads), 0, s, 1, logits, T, E, k_max, delta, idx,
+                                  gate, n_sel);
   if (err != cudaSuccess || token_offsets == nullptr) return err;
   if (n_sel == nullptr) return cudaErrorInvalidValue;
-  k_token_offsets<<<1, kScanT, 0, s>>>(n_sel, T, token_offsets);
-  return cudaGetLastError();
+  return launch_kernel(k_token_offsets, dim3(1), dim3(kScanT), 0, s, 1,
+                       static_cast<const int32_t*>(n_sel), T, token_offsets);
 }
 
 }  // namespace moe

@@ -25,6 +25,7 @@ constexpr int kStatsWarps = kStatsThreads / 32;
 __global__ void __launch_bounds__(kStatsThreads)
     k_route_prob_tiles(const float* __restrict__ logits, int T, int E, float* __restrict__ tile_prob) {
   __shared__ float part[kStatsWarps][kMaxE];
+  pdl_wait_and_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kStatsBT;
   float acc[kMaxE / 32];
@@ -77,6 +78,7 @@ __global__ void k_route_stats_reduce(const int* __restrict__ tile_counts, int co
                                      const float* __restrict__ tile_prob, int prob_tiles, int T,
                                      int E, int32_t* __restrict__ counts,
                                      float* __restrict__ prob_mean) {
+  pdl_wait_and_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
     for (int j = 0; j < count_tiles; ++j) c += tile_counts[static_cast<size_t>(j) * E + e];
@@ -91,12 +93,11 @@ cudaError_t launch_route_stats(const float* logits, const int* tile_counts, int 
                                int E, float* tile_prob, int32_t* counts, float* prob_mean,
                                cudaStream_t s) {
   const int prob_tiles = (T + kStatsBT - 1) / kStatsBT;
-  k_route_prob_tiles<<<prob_tiles, kStatsThreads, 0, s>>>(logits, T, E, tile_prob);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_kernel(k_route_prob_tiles, dim3(prob_tiles), dim3(kStatsThreads), 0, s,
+                                  1, logits, T, E, tile_prob);
   if (err != cudaSuccess) return err;
-  k_route_stats_reduce<<<1, 256, 0, s>>>(tile_counts, count_tiles, tile_prob, prob_tiles, T, E,
-                                          counts, prob_mean);
-  return cudaGetLastError();
+  return launch_kernel(k_route_stats_reduce, dim3(1), dim3(256), 0, s, 1, tile_counts, count_tiles,
+                       static_cast<const float*>(tile_prob), prob_tiles, T, E, counts, prob_mean);
 }
 
 }  // namespace moe
