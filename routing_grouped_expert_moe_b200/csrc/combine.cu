@@ -17,6 +17,49 @@ namespace moe {
 
 constexpr int kCombineThreads = 256;
 
+// One output vector: the kept slots' rows weighted by their gates, summed by
+// FMA in slot order in fp32, rounded once to the storage type.
+template <bool BF16>
+__device__ __forceinline__ void combine_store(const int4 (&q)[kMaxTopK],
+                                              const int (&rows)[kMaxTopK],
+                                              const float (&g)[kMaxTopK], uint8_t* dst) {
+  constexpr int EPV = BF16 ? 8 : 4;
+  float acc[EPV];
+#pragma unroll
+  for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxTopK; ++s) {
+    if (rows[s] < 0) continue;
+    if constexpr (BF16) {
+      const uint32_t w[4] = {static_cast<uint32_t>(q[s].x), static_cast<uint32_t>(q[s].y),
+                             static_cast<uint32_t>(q[s].z), static_cast<uint32_t>(q[s].w)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(g[s], bf16_lo(w[i]), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(g[s], bf16_hi(w[i]), acc[2 * i + 1]);
+      }
+    } else {
+      acc[0] = fmaf(g[s], __int_as_float(q[s].x), acc[0]);
+      acc[1] = fmaf(g[s], __int_as_float(q[s].y), acc[1]);
+      acc[2] = fmaf(g[s], __int_as_float(q[s].z), acc[2]);
+      acc[3] = fmaf(g[s], __int_as_float(q[s].w), acc[3]);
+    }
+  }
+  int4 o;
+  if constexpr (BF16) {
+    o.x = static_cast<int>(pack_bf16x2(acc[0], acc[1]));
+    o.y = static_cast<int>(pack_bf16x2(acc[2], acc[3]));
+    o.z = static_cast<int>(pack_bf16x2(acc[4], acc[5]));
+    o.w = static_cast<int>(pack_bf16x2(acc[6], acc[7]));
+  } else {
+    o.x = __float_as_int(acc[0]);
+    o.y = __float_as_int(acc[1]);
+    o.z = __float_as_int(acc[2]);
+    o.w = __float_as_int(acc[3]);
+  }
+  *reinterpret_cast<int4*>(dst) = o;
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kCombineThreads)
     k_combine(const uint8_t* __restrict__ y, const float* __restrict__ gate,
@@ -35,44 +78,27 @@ __global__ void __launch_bounds__(kCombineThreads)
       rows[s] = s < k ? __ldg(row_map + static_cast<size_t>(t) * k + s) : -1;
       g[s] = s < k ? (gate ? __ldg(gate + static_cast<size_t>(t) * k + s) : 1.f) : 0.f;
     }
-    for (int v = lane; v < nvec; v += 32) {
-      float acc[EPV];
-#pragma unroll
-      for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
+    // two 16-byte vectors per lane and round: every load of both is in flight
+    // before the first FMA
+    for (int v0 = lane; v0 < nvec; v0 += 64) {
+      const int v1 = v0 + 32;
+      const bool two = v1 < nvec;
+      int4 qa[kMaxTopK], qb[kMaxTopK];
 #pragma unroll
       for (int s = 0; s < kMaxTopK; ++s) {
+        qa[s] = make_int4(0, 0, 0, 0);
+        qb[s] = make_int4(0, 0, 0, 0);
         if (rows[s] < 0) continue;
-        const int4 q = __ldg(reinterpret_cast<const int4*>(
-            y + (static_cast<size_t>(rows[s]) * H + static_cast<size_t>(v) * EPV) * EB));
-        if constexpr (BF16) {
-          const uint32_t w[4] = {static_cast<uint32_t>(q.x), static_cast<uint32_t>(q.y),
-                                 static_cast<uint32_t>(q.z), static_cast<uint32_t>(q.w)};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = fmaf(g[s], bf16_lo(w[i]), acc[2 * i]);
-            acc[2 * i + 1] = fmaf(g[s], bf16_hi(w[i]), acc[2 * i + 1]);
-          }
-        } else {
-          acc[0] = fmaf(g[s], __int_as_float(q.x), acc[0]);
-          acc[1] = fmaf(g[s], __int_as_float(q.y), acc[1]);
-          acc[2] = fmaf(g[s], __int_as_float(q.z), acc[2]);
-          acc[3] = fmaf(g[s], __int_as_float(q.w), acc[3]);
-        }
+        const uint8_t* yr = y + static_cast<size_t>(rows[s]) * H * EB;
+        qa[s] = __ldg(reinterpret_cast<const int4*>(yr + static_cast<size_t>(v0) * EPV * EB));
+        if (two)
+          qb[s] = __ldg(reinterpret_cast<const int4*>(yr + static_cast<size_t>(v1) * EPV * EB));
       }
-      int4 o;
-      if constexpr (BF16) {
-        o.x = static_cast<int>(pack_bf16x2(acc[0], acc[1]));
-        o.y = static_cast<int>(pack_bf16x2(acc[2], acc[3]));
-        o.z = static_cast<int>(pack_bf16x2(acc[4], acc[5]));
-        o.w = static_cast<int>(pack_bf16x2(acc[6], acc[7]));
-      } else {
-        o.x = __float_as_int(acc[0]);
-        o.y = __float_as_int(acc[1]);
-        o.z = __float_as_int(acc[2]);
-        o.w = __float_as_int(acc[3]);
-      }
-      *reinterpret_cast<int4*>(out + (static_cast<size_t>(t) * H + static_cast<size_t>(v) * EPV) *
-                                         EB) = o;
+      combine_store<BF16>(qa, rows, g,
+                          out + (static_cast<size_t>(t) * H + static_cast<size_t>(v0) * EPV) * EB);
+      if (two)
+        combine_store<BF16>(qb, rows, g,
+                            out + (static_cast<size_t>(t) * H + static_cast<size_t>(v1) * EPV) * EB);
     }
   }
 }

@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
-    uint8_t* stg = smem + G_STAGES * G_STAGE_BYTES + (warp - 2) * 1 * G_STG_BYTES;  // this warp's staging boxes
+    // this warp's staging box
+    uint8_t* stg = smem + G_STAGES * G_STAGE_BYTES + (warp - 2) * G_STG_BYTES;
     int last_box = -1;  // box of the last committed bulk store
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;

@@ -12,9 +12,10 @@
 // Roles per CTA (320 threads): warp 0 TMA producer (both CTAs; completion is
 // counted on the first CTA's full barrier), warp 1 MMA issuer (first CTA only)
 // and TMEM owner (both: the pair allocates together), warps 2-9 epilogue of the
-// CTA's own 128 TMEM lanes (two warps per lane quarter, half the columns each).  The first CTA's commits arrive on both CTAs'
-// "stage free" and "accumulator full" barriers; both CTAs' epilogues arrive on
-// the first CTA's "accumulator free" barrier.
+// CTA's own 128 TMEM lanes (two warps per lane quarter, half the columns
+// each).  The first CTA's commits arrive on both CTAs' "stage free" and
+// "accumulator full" barriers; both CTAs' epilogues arrive on the first CTA's
+// "accumulator free" barrier.
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -244,7 +245,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int q = warp & 3;             // TMEM lanes 32q .. 32q+31
     const int half = (warp - 2) >> 2;   // which half of the tile's columns
     const int row = q * 32 + lane;
-    uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES + (warp - 2) * 2 * G_STG_BYTES;  // this warp's staging boxes
+    // this warp's two staging boxes
+    uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES + (warp - 2) * 2 * G_STG_BYTES;
     int last_box = -1;  // box of the last committed bulk store
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int acc = 0;

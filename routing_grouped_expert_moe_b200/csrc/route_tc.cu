@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(R_THREADS)
           float4 acc = __ldcg(reinterpret_cast<const float4*>(base + e0));
           for (int r = 1; r < S; ++r) {  // rank order: deterministic
             const float4 p =
-                __ldcg(reinterpret_cast<const float4*>(base + static_cast<size_t>(r) * R_BT * a.E + e0));
+                __ldcg(reinterpret_cast<const float4*>(base + static_cast<size_t>(r) * R_BT * a.E +
+                                                       e0));
             acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
           }
           const float l4[4] = {acc.x, acc.y, acc.z, acc.w};
