@@ -261,6 +261,14 @@ moe_status moe_forward_threshold(const void* x, const void* w_gate, const float*
 moe_status moe_selftest_epilogue_activations(const float* z, int n, float* gelu_out,
                                              float* silu_out, moe_stream_t stream);
 
+/* Self-test hook (no counterpart on the pages): one kernel whose bounded
+ * pipeline wait can never be satisfied.  The wait gives up after its limit
+ * (1 s) and records MOE_ERR_TIMEOUT in the status word at the start of ws (at
+ * least 256 bytes) — the path every tcgen05 kernel takes when a TMA or MMA
+ * completion never arrives — and the kernel returns, leaving the context
+ * usable.  Read the result with moe_get_device_status().                    */
+moe_status moe_selftest_bounded_wait(void* ws, moe_stream_t stream);
+
 /* Synchronises `stream`, then returns the status the kernels of the last
  * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */
 moe_status moe_get_device_status(void* ws, moe_stream_t stream);

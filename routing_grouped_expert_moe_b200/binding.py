@@ -57,6 +57,7 @@ _SIGS = {
     "moe_forward_threshold": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _f, _i, _i, _p,
                                    _p, _p, _p, _sz, _p]),
     "moe_selftest_epilogue_activations": (_i, [_p, _i, _p, _p, _p]),
+    "moe_selftest_bounded_wait": (_i, [_p, _p]),
     "moe_get_device_status": (_i, [_p, _p]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
@@ -418,6 +419,11 @@ def epilogue_activations(z):
     _check(_lib.moe_selftest_epilogue_activations(_ptr(z), z.numel(), _ptr(g), _ptr(s), _stream()),
            "moe_selftest_epilogue_activations")
     return g, s
+
+
+def selftest_bounded_wait(ws):
+    """Enqueue the self-test whose bounded wait must time out (see device_status)."""
+    _check(_lib.moe_selftest_bounded_wait(_ptr(ws), _stream()), "moe_selftest_bounded_wait")
 
 
 def device_status(ws) -> int:

@@ -364,6 +364,14 @@ moe_status moe_selftest_epilogue_activations(const float* z, int n, float* gelu_
   return cuda_status(launch_epilogue_activations(z, n, gelu_out, silu_out, as_stream(stream)));
 }
 
+moe_status moe_selftest_bounded_wait(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int* status = at<int>(ws, 0);
+  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_selftest_bounded_wait(status, s));
+}
+
 size_t moe_expert_matmul_workspace_bytes(int T, int H, int I, int E, moe_dtype dt) {
   if (T < 0 || H <= 0 || I <= 0 || E <= 0) return 0;
   return matmul_ws(T, H, I, E, dt).total;

@@ -153,6 +153,10 @@ cudaError_t launch_route_threshold(const float* logits, int T, int E, int k_max,
                                    int32_t* idx, float* gate, int32_t* n_sel,
                                    int32_t* token_offsets, cudaStream_t s);
 
+// ---------------------------------------------------------------- self-tests
+// One bounded wait that can never be satisfied (records the timeout status).
+cudaError_t launch_selftest_bounded_wait(int* status, cudaStream_t s);
+
 // ---------------------------------------------------------------- misc
 // Clears the status word and n counters (the router's tickets).
 cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters = nullptr, int n = 0);
