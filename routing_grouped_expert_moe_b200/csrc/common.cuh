@@ -303,6 +303,29 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// Bounded wait for a role with slack (an epilogue warp waiting for its next
+// accumulator): between tries the warp sleeps sleep_ns, so idle warps leave
+// the issue slots of their SM sub-partition to the producer and MMA warps.
+template <bool CLUSTER>
+__device__ __forceinline__ bool mbar_wait_polite(uint64_t* bar, uint32_t parity,
+                                                 volatile int* abort_flag, int* status,
+                                                 uint32_t sleep_ns) {
+  if (CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        record_status(status, kStatusTimeout);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // TMA loads whose completion is counted on an mbarrier that may live in the
 // other CTA of the pair (mbar is a shared::cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t mbar,

@@ -23,6 +23,8 @@ constexpr int G_SMEM = G_STAGES * G_STAGE_BYTES + G_EPI_WARPS * G_STG_BYTES + 10
 constexpr uint32_t G_TMEM_COLS = 512;
 // Default L2 prefetch distance of the GEMM producers, in k-blocks (0: off).
 constexpr int kGemmPrefetchDist = 0;
+// Default sleep of an epilogue warp between polls of its accumulator barrier.
+constexpr int kEpilogueSleepNs = 1000;
 
 template <int MODE>
 struct ModeCfg {

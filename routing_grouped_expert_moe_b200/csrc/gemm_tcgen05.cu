@@ -235,7 +235,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     for (int tau = blockIdx.x; tau < total; tau += gridDim.x) {
       const TileInfo ti = decode_tile(tau, s_prefix, s_seg_start, s_seg_rows, s_mtiles, E, BN_OUT);
       int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, args.status);
+      if (lane == 0)
+        w = mbar_wait_polite<false>(&tfull_bar[acc], acc_phase, abort_flag, args.status,
+                                    args.epi_sleep_ns);
       if (!__shfl_sync(0xffffffffu, w, 0)) break;
       tc_fence_after();
       const uint32_t t_row =
@@ -332,6 +334,9 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
   GemmArgs ga = g;
   ga.pf_dist = kGemmPrefetchDist;
   if (const char* e = getenv("MOE_GEMM_PF")) ga.pf_dist = atoi(e) < 0 ? 0 : atoi(e);
+  // MOE_EPI_SLEEP=<ns> sets the epilogue warps' sleep between accumulator polls.
+  ga.epi_sleep_ns = kEpilogueSleepNs;
+  if (const char* e = getenv("MOE_EPI_SLEEP")) ga.epi_sleep_ns = atoi(e) < 0 ? 0 : atoi(e);
   // MOE_GEMM_CTAS=<n> caps the persistent grid (a measurement aid: how the
   // GEMM scales with the number of SMs it runs on).
   if (const char* e = getenv("MOE_GEMM_CTAS")) {

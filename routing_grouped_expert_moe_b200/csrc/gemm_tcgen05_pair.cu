@@ -255,7 +255,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const PairTile ti = decode_pair(tau, s_prefix, s_seg_start, s_seg_rows, s_mtiles, E, BN_OUT,
                                       static_cast<int>(rank));
       int w = 1;
-      if (lane == 0) w = mbar_wait_cluster(&tfull_bar[acc], acc_phase, abort_flag, args.status);
+      if (lane == 0)
+        w = mbar_wait_polite<true>(&tfull_bar[acc], acc_phase, abort_flag, args.status,
+                                   args.epi_sleep_ns);
       if (!__shfl_sync(0xffffffffu, w, 0)) break;
       tc_fence_after();
       const uint32_t t_row =

@@ -109,6 +109,7 @@ struct GemmArgs {
   void* out;                 // [R_max, N]
   int* status;
   int pf_dist;               // k-blocks ahead of the TMA ring to prefetch into L2 (0: off)
+  int epi_sleep_ns;          // epilogue warps' sleep between polls of the accumulator barrier
 };
 
 struct GemmTcPlan {
