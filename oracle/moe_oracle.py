@@ -341,7 +341,8 @@ def combine(y, gates, row_map, dtype: str) -> np.ndarray:
 
 
 def threshold_select(logits, k_max: int, delta=None) -> dict:
-    """Per token: p = softmax over all E (float64); keep the experts with p > delta,
+    """Per token: p = softmax over all E (the decision in float32, as the kernel
+    takes it); keep the experts with p > delta,
     largest first (ties to the lower id), at most k_max; when none exceeds delta
     the largest alone is kept.  Gates g_s = exp(l_s - l_0) / sum_kept exp(l_j - l_0).
     delta None or <= 0: the default 1/E (as the float32 the library uses).
@@ -358,11 +359,13 @@ def threshold_select(logits, k_max: int, delta=None) -> dict:
         row = [float(v) for v in lg[t]]
         order = sorted(range(E), key=lambda e: (_rank_key(row[e]), e))
         l64 = np.asarray(row, dtype=np.float64)
-        z = np.exp(l64 - np.nanmax(l64))
-        p = z / np.nansum(z)
+        # the keep/drop decision is taken in float32, the precision the kernel uses
+        l32 = lg[t].astype(np.float32)
+        z32 = np.exp(l32 - np.float32(np.nanmax(l32)), dtype=np.float32)
+        p32 = z32 / np.float32(np.nansum(z32, dtype=np.float32))
         kept = [order[0]]
         for e in order[1:k_max]:
-            if not p[e] > d:
+            if not p32[e] > np.float32(d):
                 break
             kept.append(e)
         zk = np.exp(l64[kept] - l64[kept[0]])
