@@ -19,6 +19,7 @@
 // the tile to finish (an atomic ticket) sums all S partials in rank order —
 // deterministic whichever CTA is last — then selects.
 #include <climits>
+#include <cstdlib>
 
 #include "gemm_common.cuh"
 
@@ -28,11 +29,14 @@ constexpr int R_BT = 128;          // tokens per CTA
 constexpr int R_THREADS = 192;     // producer, MMA, 4 epilogue warps
 constexpr int R_A_BYTES = R_BT * 64 * 2;
 
-template <int NPAD>
+// DEEP: one CTA per SM (token tiles x H splits fit on the SMs), so the ring
+// takes ~192 KB and keeps twice the bytes in flight; otherwise ~96 KB so two
+// CTAs share an SM.
+template <int NPAD, bool DEEP>
 struct RouteTcCfg {
   static constexpr int B_BYTES = NPAD * 64 * 2;
   static constexpr int STAGE_BYTES = R_A_BYTES + B_BYTES;
-  static constexpr int STAGES = NPAD == 64 ? 4 : (NPAD == 128 ? 3 : 2);
+  static constexpr int STAGES = (NPAD == 64 ? 4 : (NPAD == 128 ? 3 : 2)) * (DEEP ? 2 : 1);
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = NPAD;
 };
@@ -107,11 +111,11 @@ __device__ __forceinline__ void route_tc_finish(const RouteArgs& a, int tile, in
     a.tile_counts[static_cast<size_t>(tile) * a.E + i] = cnt_s[i];
 }
 
-template <int NPAD, int K>
+template <int NPAD, int K, bool DEEP>
 __global__ void __launch_bounds__(R_THREADS)
     k_route_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                const RouteArgs a, int S) {
-  using C = RouteTcCfg<NPAD>;
+  using C = RouteTcCfg<NPAD, DEEP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -304,6 +308,20 @@ __global__ void __launch_bounds__(R_THREADS)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
+static int num_sms_for_route() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// MOE_ROUTE_DEEP=0 keeps the shallow ring (a measurement aid).
+static bool route_shallow_forced() {
+  const char* e = getenv("MOE_ROUTE_DEEP");
+  return e && e[0] == '0';
+}
+
 // W_gate [H, E] as a 2-D map (E contiguous), 64 x 64 boxes, 128-byte swizzle;
 // experts beyond E read as zeros.
 static bool make_map_wgate(CUtensorMap* m, const void* base, uint64_t H, uint64_t E) {
@@ -318,14 +336,22 @@ static bool make_map_wgate(CUtensorMap* m, const void* base, uint64_t H, uint64_
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NPAD, int K>
-static cudaError_t launch_route_tc_nk(const CUtensorMap& mx, const CUtensorMap& mw,
-                                      const RouteArgs& a, int tiles, int S, cudaStream_t s) {
-  using C = RouteTcCfg<NPAD>;
-  auto kern = k_route_tc<NPAD, K>;
+template <int NPAD, int K, bool DEEP>
+static cudaError_t launch_route_tc_nkd(const CUtensorMap& mx, const CUtensorMap& mw,
+                                       const RouteArgs& a, int tiles, int S, cudaStream_t s) {
+  using C = RouteTcCfg<NPAD, DEEP>;
+  auto kern = k_route_tc<NPAD, K, DEEP>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   return launch_kernel(kern, dim3(tiles, S, 1), dim3(R_THREADS), C::SMEM, s, 1, mx, mw, a, S);
+}
+
+template <int NPAD, int K>
+static cudaError_t launch_route_tc_nk(const CUtensorMap& mx, const CUtensorMap& mw,
+                                      const RouteArgs& a, int tiles, int S, cudaStream_t s) {
+  if (tiles * S <= num_sms_for_route() && !route_shallow_forced())
+    return launch_route_tc_nkd<NPAD, K, true>(mx, mw, a, tiles, S, s);
+  return launch_route_tc_nkd<NPAD, K, false>(mx, mw, a, tiles, S, s);
 }
 
 template <int NPAD>
