@@ -90,6 +90,9 @@ __device__ __forceinline__ void reg_fence32(float (&v)[32]) {
 //   erfc(x) = t exp(-x^2 + P(t)),  t = 1 / (1 + x/2),  P a degree-9 polynomial.
 // Then Phi(z) = 1 - erfc(|x|)/2 for z >= 0 and erfc(|x|)/2 for z < 0, so the
 // negative tail keeps its relative accuracy (1 + erf(x) would cancel).
+// SiLU(z) = z / (1 + e^-z).  Both use the special-function unit's exp and
+// reciprocal and evaluate two columns per instruction.
+
 // Reciprocal by the special-function unit (about 1 ulp; denominators here are
 // at least 1, or infinite, giving 0).
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -98,28 +101,71 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-__device__ __forceinline__ float erfc_nonneg(float ax) {
-  const float t = rcp_approx(fmaf(0.5f, ax, 1.0f));
-  float p = 0.17087277f;
-  p = fmaf(p, t, -0.82215223f);
-  p = fmaf(p, t, 1.48851587f);
-  p = fmaf(p, t, -1.13520398f);
-  p = fmaf(p, t, 0.27886807f);
-  p = fmaf(p, t, -0.18628806f);
-  p = fmaf(p, t, 0.09678418f);
-  p = fmaf(p, t, 0.37409196f);
-  p = fmaf(p, t, 1.00002368f);
-  p = fmaf(p, t, -1.26551223f);
-  return t * __expf(fmaf(-ax, ax, p));
+// Packed fp32 arithmetic (two values per instruction, sm_100): the epilogue
+// evaluates its activations on pairs of columns, halving the FMA-pipe
+// instructions that compete with the producer and MMA warps for issue slots.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
 }
 
-__device__ __forceinline__ float gelu_epi(float z) {
-  const float e = erfc_nonneg(fabsf(z) * 0.70710678118654752f);
-  return z * (z >= 0.f ? fmaf(-0.5f, e, 1.0f) : 0.5f * e);
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
-// SiLU with the hardware exponential and reciprocal: z / (1 + e^-z).
-__device__ __forceinline__ float silu_epi(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// 2^x by the special-function unit.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// GELU of two values (see above): x = |z| / sqrt 2, t = 1 / (1 + x/2),
+// erfc(x) = t 2^(log2(e) (P(t) - z^2/2)), Phi = 1 - erfc/2 (z >= 0) or erfc/2.
+__device__ __forceinline__ float2 gelu_epi2(float2 z) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float2 az = make_float2(fabsf(z.x), fabsf(z.y));
+  const float2 den = ffma2(az, splat2(0.35355339059327376f), splat2(1.0f));  // 1 + |z|/(2 sqrt 2)
+  const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+  float2 p = splat2(0.17087277f);
+  p = ffma2(p, t, splat2(-0.82215223f));
+  p = ffma2(p, t, splat2(1.48851587f));
+  p = ffma2(p, t, splat2(-1.13520398f));
+  p = ffma2(p, t, splat2(0.27886807f));
+  p = ffma2(p, t, splat2(-0.18628806f));
+  p = ffma2(p, t, splat2(0.09678418f));
+  p = ffma2(p, t, splat2(0.37409196f));
+  p = ffma2(p, t, splat2(1.00002368f));
+  p = ffma2(p, t, splat2(-1.26551223f));
+  const float2 arg = ffma2(fmul2(z, z), splat2(-0.5f), p);  // P(t) - z^2/2
+  const float2 a2 = fmul2(arg, splat2(kLog2e));
+  const float2 e = fmul2(t, make_float2(ex2_approx(a2.x), ex2_approx(a2.y)));  // erfc(|z|/sqrt 2)
+  const float2 h = fmul2(e, splat2(0.5f));
+  const float2 phi = make_float2(z.x >= 0.f ? 1.0f - h.x : h.x, z.y >= 0.f ? 1.0f - h.y : h.y);
+  return fmul2(z, phi);
+}
+
+// SiLU of two values: z / (1 + 2^(-z log2 e)).
+__device__ __forceinline__ float2 silu_epi2(float2 z) {
+  const float2 a = fmul2(z, splat2(-1.4426950408889634f));
+  const float2 d = make_float2(1.0f + ex2_approx(a.x), 1.0f + ex2_approx(a.y));
+  return fmul2(z, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
 
 // Activation of one thread's 32 accumulator columns, packed to bf16 pairs.
 template <int MODE>
@@ -127,10 +173,10 @@ __device__ __forceinline__ void epilogue_pack(const float (&v)[32], const float 
                                               uint32_t (&p)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float a0 = v[2 * i], a1 = v[2 * i + 1];
-    if (MODE == 0) { a0 = gelu_epi(a0); a1 = gelu_epi(a1); }
-    if (MODE == 1) { a0 = silu_epi(a0) * u[2 * i]; a1 = silu_epi(a1) * u[2 * i + 1]; }
-    p[i] = pack_bf16x2(a0, a1);
+    float2 a = make_float2(v[2 * i], v[2 * i + 1]);
+    if (MODE == 0) a = gelu_epi2(a);
+    if (MODE == 1) a = fmul2(silu_epi2(a), make_float2(u[2 * i], u[2 * i + 1]));
+    p[i] = pack_bf16x2(a.x, a.y);
   }
 }
 

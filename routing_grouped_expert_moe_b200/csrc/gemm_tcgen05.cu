@@ -266,9 +266,16 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 __global__ void k_epilogue_activations(const float* __restrict__ z, int n, float* __restrict__ gelu,
                                        float* __restrict__ silu) {
   pdl_wait_and_trigger();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    gelu[i] = gelu_epi(z[i]);
-    silu[i] = silu_epi(z[i]);
+  // in pairs, with the same packed code the epilogue runs
+  for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
+    const float2 zz = make_float2(z[i], i + 1 < n ? z[i + 1] : 0.f);
+    const float2 g = gelu_epi2(zz), s = silu_epi2(zz);
+    gelu[i] = g.x;
+    silu[i] = s.x;
+    if (i + 1 < n) {
+      gelu[i + 1] = g.y;
+      silu[i + 1] = s.y;
+    }
   }
 }
 
