@@ -55,9 +55,10 @@ __global__ void __launch_bounds__(S_THREADS)
     const int m0 = s_start[e] + mtile * S_BM;
     const int rows = min(S_BM, s_rows[e] - mtile * S_BM);
     const int n0 = nt * S_BN;
-    if (threadIdx.x < S_BM) {
-      const int r = threadIdx.x < rows ? m0 + threadIdx.x : -1;
-      s_arow[threadIdx.x] = r < 0 ? -1 : (GATHER ? args.row_token[r] : r);
+    const int tid = static_cast<int>(threadIdx.x);
+    if (tid < S_BM) {
+      const int r = tid < rows ? m0 + tid : -1;
+      s_arow[tid] = r < 0 ? -1 : (GATHER ? args.row_token[r] : r);
     }
     float acc[4][4], acc3[4][4];
 #pragma unroll
