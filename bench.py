@@ -217,10 +217,11 @@ def oracle_threads() -> int:
 
 
 def calibrate_tokens(cfg, d, target_s: float) -> tuple[int, float]:
+    """A token count whose oracle run takes about target_s (capped at the workload's T)."""
     n = min(cfg.T, 64)
     dt = oracle_sample(cfg, d, n)
-    while dt < 0.25 * target_s and n < cfg.T:
-        n = min(cfg.T, max(n * 2, int(n * target_s / max(dt, 1e-3) * 0.5)))
+    while dt < 0.8 * target_s and n < cfg.T:
+        n = min(cfg.T, max(n * 2, int(n * target_s / max(dt, 1e-3))))
         dt = oracle_sample(cfg, d, n)
     return n, dt
 
