@@ -121,7 +121,9 @@ def algorithmic_work(cfg: synth.MoEConfig, counts) -> dict:
     gemm2_bytes = active * H * F * s + R * F * s + R * H * s
     route_bytes = T * H * s + H * E * s + T * k * 8 + (E * 4 if cfg.bias != "none" else 0)
     scan_bytes = 2 * (E + 1) * 4
-    scatter_bytes = T * k * 4 + R * 4 + T * k * 4 + (2 * R * H * s)   # ids, row_token, row_map, x_perm
+    # ids in, row_token and row_map out, x read once, x_perm written (a token's
+    # second kept row re-reads the same x row, which the count does not repeat)
+    scatter_bytes = T * k * 4 + R * 4 + T * k * 4 + T * H * s + R * H * s
     combine_bytes = R * H * s + T * k * 8 + T * H * s
     return {"R": R, "active_experts": active, "gemm_flops": gemm_flops, "gemm1_flops": gemm1_flops,
             "gemm2_flops": gemm2_flops, "weight_bytes": weight_bytes, "gemm1_bytes": gemm1_bytes,
