@@ -185,6 +185,32 @@ moe_status moe_forward_host(const void* x_host, const void* w_gate, const float*
                             moe_act act, moe_dtype dt, void* out_host,
                             void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* A run of n_batches independent layer forwards, batch i reading x_host[i]
+ * [T, H] and writing out_host[i] [T, H] (both in HOST memory, page-locked for
+ * the copies to overlap; the pointers may repeat, e.g. a ring of buffers).
+ * Each batch is one moe_forward of its own T tokens (its own capacity, its
+ * own drops); the weights are shared.  Batch i's host-to-device copy runs on
+ * copy_in, its layer on stream and its device-to-host copy on copy_out, over
+ * two device stages of x and two of out used in turn, so the copy-in of batch
+ * i+1 and the copy-out of batch i-1 overlap the layer of batch i.  Null
+ * copy streams mean `stream` (no overlap; the same results).  All work is
+ * ordered after what is already queued on `stream`, and `stream` is ordered
+ * after all of it on return: synchronise `stream` before reading out_host.
+ * ws must hold
+ * moe_forward_host_batches_workspace_bytes(...) bytes (the moe_forward
+ * workspace plus four T x H stages).  Errors as moe_forward, all detected
+ * before anything is queued; creates and destroys seven CUDA events (no
+ * device allocation).                       */
+size_t moe_forward_host_batches_workspace_bytes(int T, int H, int F, int E, int top_k,
+                                                moe_act act, moe_dtype dt);
+moe_status moe_forward_host_batches(const void* const* x_host, void* const* out_host,
+                                    int n_batches, const void* w_gate, const float* gate_bias,
+                                    const void* w1, const void* w3, const void* w2,
+                                    int T, int H, int F, int E, int top_k,
+                                    float capacity_factor, moe_act act, moe_dtype dt,
+                                    void* ws, size_t ws_bytes, moe_stream_t stream,
+                                    moe_stream_t copy_in, moe_stream_t copy_out);
+
 /* Router load statistics.  [P3] Step 4 and [P4] §5.3 name an auxiliary
  * load-balancing loss (--moe-aux-loss-coeff) but not its formula, so the
  * router's two per-expert statistics are returned instead of a loss:

@@ -48,6 +48,9 @@ _SIGS = {
                                _sz, _p, _p, _i]),
     "moe_forward_host": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i, _i, _p, _p, _sz,
                               _p]),
+    "moe_forward_host_batches_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "moe_forward_host_batches": (_i, [_p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _i,
+                                      _i, _p, _sz, _p, _p, _p]),
     "moe_route_stats_workspace_bytes": (_sz, [_i, _i]),
     "moe_route_stats": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
     "moe_expert_matmul_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
@@ -330,6 +333,58 @@ def forward_host(x_host, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0
                                  ACT[act], _dt(x_host), _ptr(out_host), _ptr(ws), ws.numel(),
                                  _stream()), "moe_forward_host")
     return out_host
+
+
+def forward_host_batches_workspace_bytes(T, H, F, E, top_k, act="swiglu",
+                                         dtype=torch.bfloat16) -> int:
+    return int(_lib.moe_forward_host_batches_workspace_bytes(
+        T, H, F, E, top_k, ACT[act], BF16 if dtype == torch.bfloat16 else F32))
+
+
+def forward_host_batches(x_hosts, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0.0,
+                         act="swiglu", out_hosts=None, ws=None, copy_streams="new"):
+    """Independent layer forwards over a list of page-locked host batches [T, H] (all the
+    same shape), copy-in / layer / copy-out overlapped on three streams.  copy_streams:
+    (copy_in, copy_out) torch streams, "new" for two fresh ones, None for no overlap.
+    Returns the list of host outputs (valid once the current stream is synchronised)."""
+    xs = list(x_hosts)
+    if not xs:
+        return []
+    for i, xh in enumerate(xs):
+        _need(xh, f"x_hosts[{i}]", dtype=xs[0].dtype, dim=2, cuda=False)
+        if xh.is_cuda:
+            raise ValueError(f"x_hosts[{i}] must be in host memory")
+        if xh.shape != xs[0].shape:
+            raise ValueError(f"x_hosts[{i}] has shape {tuple(xh.shape)}, "
+                             f"x_hosts[0] {tuple(xs[0].shape)}")
+    T, H = xs[0].shape
+    E = w_gate.shape[1]
+    F = 8 if act == "identity" else w1.shape[2]
+    if out_hosts is None:
+        out_hosts = [torch.empty_like(xh, pin_memory=True) for xh in xs]
+    outs = list(out_hosts)
+    if len(outs) != len(xs):
+        raise ValueError(f"{len(xs)} input batches but {len(outs)} outputs")
+    for i, oh in enumerate(outs):
+        _need(oh, f"out_hosts[{i}]", dtype=xs[0].dtype, dim=2, cuda=False)
+        if oh.is_cuda:
+            raise ValueError(f"out_hosts[{i}] must be in host memory")
+        if oh.shape != xs[0].shape:
+            raise ValueError(f"out_hosts[{i}] has shape {tuple(oh.shape)}")
+    if ws is None:
+        ws = alloc_workspace(forward_host_batches_workspace_bytes(T, H, F, E, top_k, act,
+                                                                  xs[0].dtype), w_gate.device)
+    if copy_streams == "new":
+        copy_streams = (torch.cuda.Stream(w_gate.device), torch.cuda.Stream(w_gate.device))
+    cin, cout = (None, None) if copy_streams is None else copy_streams
+    xp = (ctypes.c_void_p * len(xs))(*[xh.data_ptr() for xh in xs])
+    op = (ctypes.c_void_p * len(outs))(*[oh.data_ptr() for oh in outs])
+    _check(_lib.moe_forward_host_batches(
+        xp, op, len(xs), _ptr(w_gate), _ptr(gate_bias), _ptr(w1), _ptr(w3), _ptr(w2), T, H, F,
+        E, top_k, ctypes.c_float(capacity_factor), ACT[act], _dt(xs[0]), _ptr(ws), ws.numel(),
+        _stream(), None if cin is None else cin.cuda_stream,
+        None if cout is None else cout.cuda_stream), "moe_forward_host_batches")
+    return outs
 
 
 def route_stats(x, w_gate, gate_bias=None, top_k=2, ws=None):

@@ -440,12 +440,12 @@ struct Gating {
   int32_t* n_sel_out = nullptr;
 };
 
-moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bias, const void* w1,
-                        const void* w3, const void* w2, int T, int H, int F, int E, int top_k,
-                        float capacity_factor, moe_act act, moe_dtype dt, void* out,
-                        int32_t* topk_idx_out, int32_t* expert_counts_out, void* ws,
-                        size_t ws_bytes, moe_stream_t stream, cudaEvent_t const* ev,
-                        const Gating& gating = Gating()) {
+// Every host-side check of a layer forward, in order.  MOE_OK with T == 0
+// means there is nothing to launch.
+moe_status check_forward(const void* x, const void* w_gate, const void* w1, const void* w3,
+                         const void* w2, int T, int H, int F, int E, int top_k, moe_act act,
+                         moe_dtype dt, const void* out, const void* ws, size_t ws_bytes,
+                         bool threshold) {
   moe_status st = check_common(T, H, E, top_k, dt);
   if (st != MOE_OK) return st;
   if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU && act != MOE_ACT_IDENTITY)
@@ -460,9 +460,22 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   }
   if (!index_range_ok(T, top_k, H > F ? H : F) || !index_range_ok(T, 1, E))
     return MOE_ERR_UNSUPPORTED;
-  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false, gating.threshold);
   if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return MOE_ERR_INVALID_ARG;
-  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(T, H, F, E, top_k, act, dt, false, threshold).total)
+    return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bias, const void* w1,
+                        const void* w3, const void* w2, int T, int H, int F, int E, int top_k,
+                        float capacity_factor, moe_act act, moe_dtype dt, void* out,
+                        int32_t* topk_idx_out, int32_t* expert_counts_out, void* ws,
+                        size_t ws_bytes, moe_stream_t stream, cudaEvent_t const* ev,
+                        const Gating& gating = Gating()) {
+  moe_status st = check_forward(x, w_gate, w1, w3, w2, T, H, F, E, top_k, act, dt, out, ws,
+                                ws_bytes, gating.threshold);
+  if (st != MOE_OK || T == 0) return st;
+  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false, gating.threshold);
 
   cudaStream_t s = as_stream(stream);
   const int nsm = num_sms_current();
@@ -626,6 +639,98 @@ moe_status moe_forward_host(const void* x_host, const void* w_gate, const float*
                    od, nullptr, nullptr, ws, L.x_stage, stream);
   if (st != MOE_OK) return st;
   return cuda_status(cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+// A run of independent batches with host x / out.  Device memory: the
+// forward's own workspace, then two x stages and two out stages used in turn,
+// so batch i's copy-in, batch i-1's layer and batch i-2's copy-out can run at
+// the same time on three streams.  Seven events (created and destroyed here):
+// `start` orders the copy streams after earlier work on `stream`; six order
+// the reuse of each stage:
+//   loaded[b]  copy-in of the batch in stage b done    -> its layer may start
+//   done[b]    layer of the batch in stage b done       -> its copy-out may start,
+//                                                          and stage b's x is free
+//   drained[b] copy-out of the batch in stage b done    -> stage b's out is free
+// cudaStreamWaitEvent binds to the event's latest record at the time of the
+// call, and the host issues batch i's three steps in order, so each wait
+// refers to the batch two steps earlier.
+size_t moe_forward_host_batches_workspace_bytes(int T, int H, int F, int E, int top_k,
+                                                moe_act act, moe_dtype dt) {
+  if (T < 0 || H <= 0 || F <= 0 || E <= 0 || top_k <= 0) return 0;
+  const size_t stage = align_up(static_cast<size_t>(T) * H * elem_bytes(dt));
+  return ws_layout(T, H, F, E, top_k, act, dt, false).total + 4 * stage;
+}
+
+moe_status moe_forward_host_batches(const void* const* x_host, void* const* out_host,
+                                    int n_batches, const void* w_gate, const float* gate_bias,
+                                    const void* w1, const void* w3, const void* w2, int T, int H,
+                                    int F, int E, int top_k, float capacity_factor, moe_act act,
+                                    moe_dtype dt, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream, moe_stream_t copy_in,
+                                    moe_stream_t copy_out) {
+  moe_status st = check_common(T, H, E, top_k, dt);
+  if (st != MOE_OK) return st;
+  if (n_batches < 0 || F <= 0 || F % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0 || n_batches == 0) return MOE_OK;
+  if (!x_host || !out_host || !ws) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_batches; ++i)
+    if (!x_host[i] || !out_host[i]) return MOE_ERR_INVALID_ARG;
+  const size_t fwd = ws_layout(T, H, F, E, top_k, act, dt, false).total;
+  const size_t bytes = static_cast<size_t>(T) * H * elem_bytes(dt);
+  const size_t stage = align_up(bytes);
+  void* xs[2] = {at<void>(ws, fwd), at<void>(ws, fwd + stage)};
+  void* os[2] = {at<void>(ws, fwd + 2 * stage), at<void>(ws, fwd + 3 * stage)};
+  // every check the batches' forwards will make, before anything is queued
+  st = check_forward(xs[0], w_gate, w1, w3, w2, T, H, F, E, top_k, act, dt, os[0], ws, fwd, false);
+  if (st != MOE_OK) return st;
+  if (ws_bytes < fwd + 4 * stage) return MOE_ERR_WORKSPACE;
+  cudaStream_t sc = as_stream(stream);
+  cudaStream_t si = copy_in ? as_stream(copy_in) : sc;
+  cudaStream_t so = copy_out ? as_stream(copy_out) : sc;
+
+  cudaEvent_t ev[7] = {};  // start, loaded[2], done[2], drained[2]
+  for (int i = 0; i < 7; ++i) {
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return MOE_ERR_CUDA;
+    }
+  }
+  cudaEvent_t start = ev[0], *loaded = ev + 1, *done = ev + 3, *drained = ev + 5;
+  auto run = [&]() -> moe_status {
+    // the copy streams start after everything already queued on `stream`
+    if (cudaEventRecord(start, sc) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(si, start, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(so, start, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int i = 0; i < n_batches; ++i) {
+      const int b = i & 1;
+      if (i >= 2 && cudaStreamWaitEvent(si, done[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaMemcpyAsync(xs[b], x_host[i], bytes, cudaMemcpyHostToDevice, si) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaEventRecord(loaded[b], si) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaStreamWaitEvent(sc, loaded[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+      if (i >= 2 && cudaStreamWaitEvent(sc, drained[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+      const moe_status s = moe_forward(xs[b], w_gate, gate_bias, w1, w3, w2, T, H, F, E, top_k,
+                                       capacity_factor, act, dt, os[b], nullptr, nullptr, ws, fwd,
+                                       stream);
+      if (s != MOE_OK) return s;
+      if (cudaEventRecord(done[b], sc) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaStreamWaitEvent(so, done[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaMemcpyAsync(out_host[i], os[b], bytes, cudaMemcpyDeviceToHost, so) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaEventRecord(drained[b], so) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  };
+  st = run();
+  // `stream` ends after everything issued on the copy streams, also when a
+  // step above failed part-way
+  if (cudaEventRecord(loaded[0], si) != cudaSuccess ||
+      cudaStreamWaitEvent(sc, loaded[0], 0) != cudaSuccess ||
+      cudaEventRecord(drained[0], so) != cudaSuccess ||
+      cudaStreamWaitEvent(sc, drained[0], 0) != cudaSuccess)
+    st = st == MOE_OK ? MOE_ERR_CUDA : st;
+  for (int i = 0; i < 7; ++i) cudaEventDestroy(ev[i]);  // released once their work completes
+  return st;
 }
 
 moe_status moe_get_device_status(void* ws, moe_stream_t stream) {

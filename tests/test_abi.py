@@ -128,3 +128,25 @@ def test_route_stats_and_expert_matmul_reject_on_host():
     assert mm(ws_bytes=mneed - 1) == B.ERR_WORKSPACE
     assert mm(w=MISALIGNED) == B.ERR_INVALID_ARG
     assert mm(T=0) == B.OK
+
+
+def test_host_batches_rejects_on_host():
+    L = B._lib
+    need = L.moe_forward_host_batches_workspace_bytes(64, 128, 256, 4, 2, 0, 1)
+    base = L.moe_workspace_bytes(64, 128, 256, 4, 2, 0, 1)
+    assert need == base + 4 * 64 * 128 * 2 and need % 256 == 0
+    assert L.moe_forward_host_batches_workspace_bytes(64, 128, 0, 4, 2, 0, 1) == 0
+    ptrs = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    holes = (ctypes.c_void_p * 2)(0x10000, None)
+
+    def call(n=2, xs=ptrs, outs=ptrs, k=2, ws_bytes=need, F=256):
+        return L.moe_forward_host_batches(xs, outs, n, FAKE, None, FAKE, FAKE, FAKE, 64, 128, F, 4,
+                                          k, ctypes.c_float(0), 0, 1, FAKE, ws_bytes, None, None,
+                                          None)
+    assert call(ws_bytes=need - 1) == B.ERR_WORKSPACE
+    assert call(n=-1) == B.ERR_INVALID_ARG
+    assert call(n=0) == B.OK                                                 # nothing to do
+    assert call(xs=holes) == B.ERR_INVALID_ARG                               # a null batch
+    assert call(outs=None) == B.ERR_INVALID_ARG
+    assert call(k=5) == B.ERR_INVALID_ARG                                    # top_k > E
+    assert call(F=100) == B.ERR_INVALID_ARG

@@ -133,6 +133,32 @@ def test_forward_deterministic_and_host_entry_point():
     assert torch.equal(oh, o1.cpu())
 
 
+@pytest.mark.parametrize("overlap", [True, False], ids=["three_streams", "one_stream"])
+def test_host_batches_equal_one_forward_per_batch(overlap):
+    """Pipelined host batches (two device stages reused in turn) give, for every
+    batch, exactly what one moe_forward of that batch gives; batches 5 and 6
+    repeat the host buffers of batches 0 and 1."""
+    cfg = _small_cfg("page1_gelu", name="batches", T=4096, H=1024, F=2048, seed=2025)
+    d = synth.make_inputs(cfg)
+    g = _cuda(d)
+    xs = [synth.normal(2025 + i, synth.STREAM_X, (cfg.T, cfg.H), 1.0, torch.bfloat16).pin_memory()
+          for i in range(5)]
+    xs += xs[:2]
+    outs = [torch.empty_like(x, pin_memory=True) for x in xs]
+    got = B().forward_host_batches(xs, g["w_gate"], g["gate_bias"], g["w1"], None, g["w2"],
+                                   cfg.top_k, cfg.capacity_factor, cfg.act, out_hosts=outs,
+                                   copy_streams="new" if overlap else None)
+    torch.cuda.synchronize()
+    ws = B().alloc_workspace(B().workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k, cfg.act,
+                                                 cfg.torch_dtype))
+    for i, x in enumerate(xs):
+        ref = B().forward(x.cuda(), g["w_gate"], g["gate_bias"], g["w1"], None, g["w2"],
+                          cfg.top_k, cfg.capacity_factor, cfg.act, ws=ws)
+        assert torch.equal(got[i], ref.cpu()), i
+    assert B().device_status(ws) == B().OK
+    assert torch.equal(got[5], got[0]) and not torch.equal(got[0], got[1])
+
+
 def test_forward_empty_and_one_token():
     cfg = _small_cfg("mixtral_e8", name="one", T=1, H=256, F=256, seed=2030)
     d = synth.make_inputs(cfg)
