@@ -143,7 +143,9 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
  * outputs); [P3] SparseScatterAdd; [P4] §4 (npu_moe_token_postprocess).
  *   out[t] = sum_{s=0..k-1, row_map[t,s] >= 0} topk_gate[t,s] * y[row_map[t,s]]
  * summed in slot order in fp32 and rounded once to dt; no atomics, so the
- * result is bit-identical from run to run.                                  */
+ * result is bit-identical from run to run.  topk_gate may be NULL: every
+ * weight is 1, and with top_k = 1 the call is a plain row gather
+ * out[t] = y[row_map[t,0]] (exact; zero where row_map is -1).               */
 moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
                                  int T, int H, int top_k, moe_dtype dt, void* out,
                                  moe_stream_t stream);

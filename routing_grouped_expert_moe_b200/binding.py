@@ -255,8 +255,10 @@ def grouped_ffn(expert_offsets, w1, w3, w2, act="swiglu", x_perm=None, x=None, r
 
 
 def unpermute_combine(y, topk_gate, row_map, out=None):
+    """out[t] = sum_s topk_gate[t,s] * y[row_map[t,s]]; topk_gate None means weights of 1."""
     _need(y, "y", dim=2)
-    _need(topk_gate, "topk_gate", dtype=torch.float32, dim=2)
+    if topk_gate is not None:
+        _need(topk_gate, "topk_gate", dtype=torch.float32, dim=2)
     _need(row_map, "row_map", dtype=torch.int32, dim=2)
     T, k = row_map.shape
     H = y.shape[1]

@@ -285,8 +285,7 @@ moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const in
   if (T < 0 || H <= 0 || top_k <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
   if (top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
-  if (!y || !topk_gate || !row_map || !out || !aligned16(y) || !aligned16(out))
-    return MOE_ERR_INVALID_ARG;
+  if (!y || !row_map || !out || !aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (!index_range_ok(T, top_k, H)) return MOE_ERR_UNSUPPORTED;
   return cuda_status(launch_combine(y, topk_gate, row_map, T, H, top_k, dt == MOE_BF16, out,
                                     num_sms_current(), as_stream(stream)));

@@ -1,0 +1,154 @@
+"""Expert-parallel forward of the MoE layer: one process per GPU, rank r of G
+owning experts [r*E/G, (r+1)*E/G).
+
+"ops-transformer 算子精讲：昇腾 NPU 上的注意力机制与融合算子实现" ch.5: with the
+experts spread over devices, routing costs two all-to-all exchanges, one that
+sends each token's hidden state to the devices of its chosen experts and one
+that brings the expert outputs back.  "ops-transformer 仓库 - MoE 算子优化实战"
+§2 (sparse computation): expert parallelism, with one aggregated all-to-all
+instead of point-to-point messages.
+
+Every rank runs the layer on its own tokens (its own capacity and drops, as
+one single-device call would) and the results equal, row for row, what one
+single-device forward of those tokens over all E experts gives:
+
+  1. route and permute the local tokens over all E experts (the permuted rows
+     come out grouped by expert, hence by owning rank);
+  2. exchange the per-expert kept-row counts (all-to-all, E/G int32 per pair);
+  3. exchange the rows (all-to-all with per-rank splits); the received block
+     is ordered [source rank][local expert];
+  4. regroup it by local expert (a k = 1 permute, stable, so sources stay in
+     rank order inside an expert), run the grouped FFN, and put the outputs
+     back in received order (a k = 1 unpermute);
+  5. the reverse all-to-all returns each output row to the rank and the row
+     slot its input came from, and the local combine sums the gated rows.
+
+Rows travel as raw bytes, so any storage type crosses unchanged.  The split
+sizes are read on the host (one device-to-host read of the offsets, one of
+the received counts): all-to-all with uneven splits needs them there.
+
+The per-rank compute steps are the C ABI's kernels (`CudaSteps`); torch.distributed
+(NCCL between GPUs) carries the two exchanges.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+def split_rows(offsets: np.ndarray, world: int) -> np.ndarray:
+    """Rows of the expert-ordered block destined to each rank: rank d owns experts
+    [d*E/G, (d+1)*E/G), whose rows run from offsets[d*E/G] to offsets[(d+1)*E/G]."""
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E = offsets.size - 1
+    if E % world:
+        raise ValueError(f"{E} experts do not split evenly over {world} ranks")
+    el = E // world
+    return np.array([offsets[(d + 1) * el] - offsets[d * el] for d in range(world)],
+                    dtype=np.int64)
+
+
+def local_expert_ids(recv_kept: np.ndarray) -> np.ndarray:
+    """Local expert id of every received row.  recv_kept[s, j] rows of local expert j
+    arrive from source rank s, sources in rank order, experts in order inside each."""
+    recv_kept = np.asarray(recv_kept, dtype=np.int64)
+    G, el = recv_kept.shape
+    return np.repeat(np.tile(np.arange(el, dtype=np.int32), G), recv_kept.reshape(-1))
+
+
+class CudaSteps:
+    """The per-rank compute steps, each one call into the C ABI on the current stream."""
+
+    def __init__(self):
+        from routing_grouped_expert_moe_b200 import binding
+        self.B = binding
+
+    def route(self, x, w_gate, gate_bias, top_k):
+        return self.B.route(x, w_gate, gate_bias, top_k)
+
+    def permute(self, x, idx, E, capacity_factor):
+        p = self.B.permute(idx, E, capacity_factor, x=x)
+        return p["x_perm"], p["offsets"], p["row_map"]
+
+    def grouped_ffn(self, x_rows, offsets, w1, w3, w2, act):
+        return self.B.grouped_ffn(offsets, w1, w3, w2, act, x_perm=x_rows)
+
+    def unpermute(self, y, row_map):
+        return self.B.unpermute_combine(y, None, row_map)
+
+    def combine(self, y, gate, row_map):
+        return self.B.unpermute_combine(y, gate, row_map)
+
+    def to_host(self, t):
+        return t.cpu().numpy()
+
+    def from_host(self, a, like):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(like.device)
+
+
+def _bytes(t: torch.Tensor) -> torch.Tensor:
+    """The rows of a contiguous [n, H] tensor as [n, H * element size] bytes."""
+    return t.view(torch.uint8)
+
+
+def ep_forward(x, w_gate, gate_bias, w1_local, w3_local, w2_local, top_k: int,
+               capacity_factor: float, act: str, num_experts: int, group=None, steps=None):
+    """The layer's output [T, H] for this rank's tokens x [T, H].
+
+    w_gate [H, E] (and gate_bias [E]) are the whole router, the same on every
+    rank; w1_local / w3_local [E/G, H, F] and w2_local [E/G, F, H] are this rank's
+    experts (w3_local None for GELU).  Every rank of `group` must call this
+    together with the same E, top_k, act and storage type (T may differ)."""
+    steps = steps or CudaSteps()
+    G = dist.get_world_size(group)
+    E = int(num_experts)
+    if E % G:
+        raise ValueError(f"{E} experts do not split evenly over {G} ranks")
+    el = E // G
+    if w1_local is not None and w1_local.shape[0] != el:
+        raise ValueError(f"w1_local holds {w1_local.shape[0]} experts, expected {el}")
+    T, H = x.shape
+    dev = x.device
+
+    # 1. route and permute this rank's tokens over all E experts
+    if T > 0:
+        idx, gate = steps.route(x, w_gate, gate_bias, top_k)
+        x_perm, offsets_d, row_map = steps.permute(x, idx, E, capacity_factor)
+        offsets = steps.to_host(offsets_d).astype(np.int64)
+    else:
+        gate = row_map = None
+        x_perm = x.new_empty(0, H)
+        offsets = np.zeros(E + 1, dtype=np.int64)
+    send = split_rows(offsets, G)
+    R = int(offsets[E])
+
+    # 2. kept-row counts per (destination, expert)
+    kept = torch.from_numpy(np.diff(offsets).astype(np.int32)).to(dev)
+    recv_kept_d = torch.empty(E, dtype=torch.int32, device=dev)
+    dist.all_to_all_single(recv_kept_d, kept, group=group)
+    recv_kept = steps.to_host(recv_kept_d).astype(np.int64).reshape(G, el)
+    recv = recv_kept.sum(axis=1)
+    R_in = int(recv.sum())
+
+    # 3. the rows, to the ranks that own their experts
+    x_in = x.new_empty(R_in, H)
+    dist.all_to_all_single(_bytes(x_in), _bytes(x_perm[:R]), output_split_sizes=recv.tolist(),
+                           input_split_sizes=send.tolist(), group=group)
+
+    # 4. regroup by local expert, run the experts, restore the received order
+    if R_in > 0:
+        ids = steps.from_host(local_expert_ids(recv_kept).reshape(R_in, 1), x_in)
+        x_loc, off_loc, map_loc = steps.permute(x_in, ids, el, 0.0)
+        y_loc = steps.grouped_ffn(x_loc, off_loc, w1_local, w3_local, w2_local, act)
+        y_in = steps.unpermute(y_loc, map_loc)
+    else:
+        y_in = x.new_empty(0, H)
+
+    # 5. outputs back to the rows they came from, then the gated sum per token
+    y_back = x.new_empty(max(R, 1), H)
+    dist.all_to_all_single(_bytes(y_back[:R]), _bytes(y_in), output_split_sizes=send.tolist(),
+                           input_split_sizes=recv.tolist(), group=group)
+    if T == 0:
+        return x.new_empty(0, H)
+    return steps.combine(y_back, gate, row_map)
