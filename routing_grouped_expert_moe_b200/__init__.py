@@ -5,11 +5,13 @@ grouped expert FFN (tcgen05 / TMEM GEMMs) -> deterministic combine, all in
 hand-written sm_100a kernels behind a C ABI (``include/moe_b200.h``).
 
 The ops live in :mod:`routing_grouped_expert_moe_b200.binding`; importing them
-loads ``lib/libmoe_b200.so`` and raises if it has not been built.
+loads ``lib/libmoe_b200.so`` and raises if it has not been built.  The
+expert-parallel forward over a torch.distributed group is in
+:mod:`routing_grouped_expert_moe_b200.expert_parallel`.
 """
 import importlib
 
-__all__ = ["binding", "synth"]
+__all__ = ["binding", "expert_parallel", "synth"]
 
 
 def __getattr__(name):
