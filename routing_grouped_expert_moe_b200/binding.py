@@ -348,7 +348,8 @@ def forward_host_batches(x_hosts, w_gate, gate_bias, w1, w3, w2, top_k, capacity
     """Independent layer forwards over a list of page-locked host batches [T, H] (all the
     same shape), copy-in / layer / copy-out overlapped on three streams.  copy_streams:
     (copy_in, copy_out) torch streams, "new" for two fresh ones, None for no overlap.
-    Returns the list of host outputs (valid once the current stream is synchronised)."""
+    Returns the list of host outputs, valid once the current stream is synchronised; the
+    host buffers must stay alive until then (the copies are asynchronous)."""
     xs = list(x_hosts)
     if not xs:
         return []
