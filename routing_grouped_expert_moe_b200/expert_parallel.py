@@ -29,6 +29,15 @@ the received counts): all-to-all with uneven splits needs them there.
 
 The per-rank compute steps are the C ABI's kernels (`CudaSteps`); torch.distributed
 (NCCL between GPUs) carries the two exchanges.
+
+With overlap=True (and at least two experts per rank) the local experts form
+two groups, A = the first half and B = the rest, and the rows move as
+point-to-point messages per group, following the same pages' point that
+expert parallelism lets communication overlap computation: B's rows travel
+while A's experts run, and A's outputs travel back while B's experts run.  A
+group's rows for one destination are contiguous in the expert-ordered block
+(experts of a rank are consecutive), so every message is a slice of an
+existing buffer; a rank's rows for itself are copied locally.
 """
 from __future__ import annotations
 
@@ -92,14 +101,88 @@ def _bytes(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.uint8)
 
 
+def _post(sends, recvs, me, group, tag):
+    """Start one point-to-point round: sends[p] goes to rank p, recvs[p] is filled by
+    rank p (contiguous byte views, None when empty: both sides derive the same sizes
+    from the exchanged counts, so they skip the same messages).  The block for this
+    rank itself is copied locally.  Returns the pending requests."""
+    ops = []
+    for peer, (snd, rcv) in enumerate(zip(sends, recvs)):
+        if peer == me:
+            if rcv is not None:
+                rcv.copy_(snd)
+            continue
+        gpeer = peer if group is None else dist.get_global_rank(group, peer)
+        if snd is not None:
+            ops.append(dist.P2POp(dist.isend, snd, gpeer, group, tag))
+        if rcv is not None:
+            ops.append(dist.P2POp(dist.irecv, rcv, gpeer, group, tag))
+    return dist.batch_isend_irecv(ops) if ops else []
+
+
+def _wait(works):
+    for w in works:
+        w.wait()
+
+
+def _rows(buf, a, b):
+    return _bytes(buf[a:b]) if b > a else None
+
+
+def _overlapped_experts(steps, x_perm, offsets, recv_kept, w1, w3, w2, act, G, el, me,
+                        group, y_back):
+    """Rows out, experts, rows back, in two expert groups that overlap (see the module
+    docstring); fills y_back (rows in the order of x_perm)."""
+    H = x_perm.shape[1]
+    halves = [(0, el // 2), (el // 2, el)]
+    recv_in = []                       # per group: [G] received row counts per source
+    bufs = []
+    pending = []
+    for gi, (j0, j1) in enumerate(halves):
+        rk = recv_kept[:, j0:j1]
+        cnt = rk.sum(axis=1)
+        starts = np.concatenate([[0], np.cumsum(cnt)])
+        buf = x_perm.new_empty(int(starts[-1]), H)
+        sends = [_rows(x_perm, int(offsets[d * el + j0]), int(offsets[d * el + j1]))
+                 for d in range(G)]
+        recvs = [_rows(buf, int(starts[s]), int(starts[s + 1])) for s in range(G)]
+        pending.append(_post(sends, recvs, me, group, tag=gi))
+        recv_in.append((rk, starts))
+        bufs.append(buf)
+    back = []
+    for gi, (j0, j1) in enumerate(halves):
+        _wait(pending[gi])             # this group's rows are here; the next may still travel
+        rk, starts = recv_in[gi]
+        buf = bufs[gi]
+        if buf.shape[0] > 0:
+            ids = steps.from_host(local_expert_ids(rk).reshape(-1, 1), buf)
+            x_loc, off_loc, map_loc = steps.permute(buf, ids, j1 - j0, 0.0)
+            sl = slice(j0, j1)
+            y_loc = steps.grouped_ffn(x_loc, off_loc, None if w1 is None else w1[sl],
+                                      None if w3 is None else w3[sl],
+                                      None if w2 is None else w2[sl], act)
+            y_in = steps.unpermute(y_loc, map_loc)
+        else:
+            y_in = buf
+        sends = [_rows(y_in, int(starts[s]), int(starts[s + 1])) for s in range(G)]
+        recvs = [_rows(y_back, int(offsets[d * el + j0]), int(offsets[d * el + j1]))
+                 for d in range(G)]
+        back.append(_post(sends, recvs, me, group, tag=2 + gi))
+    for w in back:
+        _wait(w)
+
+
 def ep_forward(x, w_gate, gate_bias, w1_local, w3_local, w2_local, top_k: int,
-               capacity_factor: float, act: str, num_experts: int, group=None, steps=None):
+               capacity_factor: float, act: str, num_experts: int, group=None, steps=None,
+               overlap: bool = False):
     """The layer's output [T, H] for this rank's tokens x [T, H].
 
     w_gate [H, E] (and gate_bias [E]) are the whole router, the same on every
     rank; w1_local / w3_local [E/G, H, F] and w2_local [E/G, F, H] are this rank's
     experts (w3_local None for GELU).  Every rank of `group` must call this
-    together with the same E, top_k, act and storage type (T may differ)."""
+    together with the same E, top_k, act, storage type and overlap (T may
+    differ).  overlap=True splits the exchanges in two expert groups so that
+    transfers overlap the expert GEMMs (needs E/G >= 2; otherwise ignored)."""
     steps = steps or CudaSteps()
     G = dist.get_world_size(group)
     E = int(num_experts)
@@ -130,6 +213,15 @@ def ep_forward(x, w_gate, gate_bias, w1_local, w3_local, w2_local, top_k: int,
     recv_kept = steps.to_host(recv_kept_d).astype(np.int64).reshape(G, el)
     recv = recv_kept.sum(axis=1)
     R_in = int(recv.sum())
+
+    if overlap and el >= 2:
+        # 3-5 in two expert groups whose transfers overlap the other group's experts
+        y_back = x.new_empty(max(R, 1), H)
+        _overlapped_experts(steps, x_perm, offsets, recv_kept, w1_local, w3_local, w2_local,
+                            act, G, el, dist.get_rank(group), group, y_back)
+        if T == 0:
+            return x.new_empty(0, H)
+        return steps.combine(y_back, gate, row_map)
 
     # 3. the rows, to the ranks that own their experts
     x_in = x.new_empty(R_in, H)

@@ -4,8 +4,9 @@ exchange logic on CPU ranks over gloo.
 The per-rank compute steps here are the oracle's (the product runs the C ABI's
 kernels in their place); what is under test is what the expert-parallel path
 adds: split sizes, the count exchange, the row exchanges both ways, the regroup
-by local expert and its inverse.  Each rank's result must equal one
-single-device oracle forward of that rank's tokens over all E experts.
+by local expert and its inverse, and the overlapped variant's point-to-point
+rounds per expert group.  Each rank's result must equal one single-device
+oracle forward of that rank's tokens over all E experts.
 """
 import os
 import socket
@@ -132,17 +133,21 @@ def _rank_main(rank: int, port: int, names, q):
             E, el = d["E"], d["E"] // WORLD
             sl = slice(rank * el, (rank + 1) * el)
             local = lambda w: None if w is None else w[sl].contiguous()  # noqa: E731
-            out = EP.ep_forward(d["x"], d["w_gate"], d["gate_bias"], local(d["w1"]),
-                                local(d["w3"]), local(d["w2"]), d["k"], d["cf"], d["act"], E,
-                                steps=OracleSteps(d["dtype"]))
-            assert out.shape == d["x"].shape and out.dtype == d["x"].dtype
+            outs = [EP.ep_forward(d["x"], d["w_gate"], d["gate_bias"], local(d["w1"]),
+                                  local(d["w3"]), local(d["w2"]), d["k"], d["cf"], d["act"], E,
+                                  steps=OracleSteps(d["dtype"]), overlap=ov)
+                    for ov in (False, True)]
+            for out in outs:
+                assert out.shape == d["x"].shape and out.dtype == d["x"].dtype
+            # the overlapped exchange moves the same rows: the same bits
+            assert torch.equal(outs[0], outs[1]), name
             if d["x"].shape[0] == 0:
                 q.put((name, rank, 0.0, 1.0))
                 continue
             f = lambda t: None if t is None else as_np(t)  # noqa: E731
             ref = O.moe_forward(f(d["x"]), f(d["w_gate"]), f(d["gate_bias"]), f(d["w1"]),
                                 f(d["w3"]), f(d["w2"]), d["k"], d["cf"], d["act"], d["dtype"])
-            got = as_np(out)
+            got = as_np(outs[1])
             same = float(np.mean(got == ref["out"]))
             q.put((name, rank, rel_err(got, ref["out"]), same))
     finally:

@@ -1,7 +1,7 @@
 """Expert-parallel forward on the GPU with one NCCL rank: every exchange runs
 (counts, rows out, rows back) through NCCL, and every compute step through the
 C ABI's kernels, including the k = 1 regroup and its inverse (the combine with
-no gates).  More ranks need more GPUs than these tests get; the exchange logic
+no gates), in both the one-round and the two-group (overlapped) form.  More ranks need more GPUs than these tests get; the exchange logic
 over several ranks is checked on CPU ranks (test_expert_parallel.py)."""
 import numpy as np
 import pytest
@@ -66,3 +66,10 @@ def test_expert_parallel_one_rank(one_rank, name, kw):
     y = B().grouped_ffn(p["offsets"], g["w1"], g["w3"], g["w2"], cfg.act, x_perm=p["x_perm"][:R])
     staged = B().unpermute_combine(y, gate, p["row_map"])
     assert torch.equal(out, staged)
+    # two expert groups (the overlapped exchange; on one rank every block is a local copy):
+    # the experts run as two grouped GEMMs, whose tile variant may differ from one GEMM's
+    ov = EP.ep_forward(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"],
+                       cfg.top_k, cfg.capacity_factor, cfg.act, cfg.E, overlap=True)
+    torch.cuda.synchronize()
+    assert rel_err(as_np(ov), ref["out"]) <= TOL[cfg.dtype]
+    assert float((ov == out).float().mean()) >= 0.999
