@@ -93,7 +93,14 @@ def _check(status: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """The tensor's address for the C ABI.  A device tensor must live on the current
+    device: the kernels run there, and another GPU's memory is not theirs to read."""
+    if t is None:
+        return None
+    if t.is_cuda and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream():
@@ -380,6 +387,10 @@ def forward_host_batches(x_hosts, w_gate, gate_bias, w1, w3, w2, top_k, capacity
     if copy_streams == "new":
         copy_streams = (torch.cuda.Stream(w_gate.device), torch.cuda.Stream(w_gate.device))
     cin, cout = (None, None) if copy_streams is None else copy_streams
+    for st in (cin, cout):
+        if st is not None and st.device.index != torch.cuda.current_device():
+            raise ValueError(f"copy stream on {st.device}, but the current device is "
+                             f"cuda:{torch.cuda.current_device()}")
     xp = (ctypes.c_void_p * len(xs))(*[xh.data_ptr() for xh in xs])
     op = (ctypes.c_void_p * len(outs))(*[oh.data_ptr() for oh in outs])
     _check(_lib.moe_forward_host_batches(
