@@ -213,8 +213,9 @@ moe_status moe_forward_host_batches(const void* const* x_host, void* const* out_
                                     void* ws, size_t ws_bytes, moe_stream_t stream,
                                     moe_stream_t copy_in, moe_stream_t copy_out);
 
-/* Router load statistics.  [P3] Step 4 and [P4] §5.3 name an auxiliary
- * load-balancing loss (--moe-aux-loss-coeff) but not its formula, so the
+/* Router load statistics.  [P3] "实战中的坑与解法" (track each expert's load)
+ * and [P4] §5.3 name an auxiliary load-balancing loss (--moe-aux-loss-coeff)
+ * but not its formula, so the
  * router's two per-expert statistics are returned instead of a loss:
  *   expert_counts[e] (int32, pre-drop) = #{(t,s): topk_idx[t,s] = e}
  *   prob_mean[e]     (fp32)            = (1/T) sum_t softmax_e(logits[t])

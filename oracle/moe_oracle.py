@@ -393,8 +393,9 @@ def moe_forward_threshold(x, w_gate, gate_bias, w1, w3, w2, k_max: int, delta,
 
 
 # --------------------------------------------------------------------------
-# Router load statistics.   [P3] Step 4 / [P4] §5.3 (auxiliary load-balancing
-# loss named, formula not given: the two per-expert statistics it is built from)
+# Router load statistics.   [P3] "实战中的坑与解法" (track each expert's load) /
+# [P4] §5.3 (auxiliary load-balancing loss named, formula not given: the two
+# per-expert statistics it is built from)
 # --------------------------------------------------------------------------
 
 

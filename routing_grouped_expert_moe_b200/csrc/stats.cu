@@ -2,10 +2,11 @@
 // probability over tokens, the two per-expert quantities a load-balancing
 // auxiliary loss is built from.
 //
-// "ops-transformer 仓库 - MoE 算子优化实战" Step 4 and lshu.cn torch_npu
-// fused-operator article §5.3 (--moe-aux-loss-coeff 0.01 against expert
-// overload) name an auxiliary load-balancing loss but not its formula, so only
-// the statistics are produced:
+// "ops-transformer 仓库 - MoE 算子优化实战", "实战中的坑与解法" (collect each
+// expert's utilisation periodically against overloaded experts) and lshu.cn
+// torch_npu fused-operator article §5.3 (--moe-aux-loss-coeff 0.01 against
+// expert overload) name the per-expert load and an auxiliary load-balancing
+// loss but not its formula, so only the statistics are produced:
 //   count[e]     = #{(t,s): topk_idx[t,s] = e}            (pre-drop)
 //   prob_mean[e] = (1/T) sum_t softmax(logits[t])[e]     (softmax over all E)
 // Both reductions run in a fixed order (tokens within a tile, then tiles), so

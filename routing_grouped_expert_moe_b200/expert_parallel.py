@@ -4,9 +4,9 @@ owning experts [r*E/G, (r+1)*E/G).
 "ops-transformer 算子精讲：昇腾 NPU 上的注意力机制与融合算子实现" ch.5: with the
 experts spread over devices, routing costs two all-to-all exchanges, one that
 sends each token's hidden state to the devices of its chosen experts and one
-that brings the expert outputs back.  "ops-transformer 仓库 - MoE 算子优化实战"
-§2 (sparse computation): expert parallelism, with one aggregated all-to-all
-instead of point-to-point messages.
+that brings the expert outputs back.  "ops-transformer 仓库 - MoE 算子优化实战",
+core principles, point 2 (sparse-computation optimisation): expert
+parallelism, with one aggregated all-to-all instead of point-to-point messages.
 
 Every rank runs the layer on its own tokens (its own capacity and drops, as
 one single-device call would) and the results equal, row for row, what one
