@@ -167,7 +167,9 @@ moe_status moe_forward(const void* x, const void* w_gate, const float* gate_bias
  * events: n_events (>= 7) cudaEvent_t handles; events[i] is recorded before
  * stage i and events[6] after the last: route (0-1), offsets scan (1-2;
  * empty: the scan runs inside the scatter kernel), scatter (2-3), expert
- * GEMM-1 (3-4), expert GEMM-2 (4-5), combine (5-6).                        */
+ * GEMM-1 (3-4), expert GEMM-2 (4-5), combine (5-6).  A NULL entry is not
+ * recorded; an event between two kernels ends their programmatic-launch
+ * overlap, so recording fewer boundaries perturbs the timing less.          */
 moe_status moe_forward_timed(const void* x, const void* w_gate, const float* gate_bias,
                              const void* w1, const void* w3, const void* w2,
                              int T, int H, int F, int E, int top_k, float capacity_factor,

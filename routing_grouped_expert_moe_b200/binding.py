@@ -310,11 +310,13 @@ def forward(x, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor=0.0, act="s
 
 def forward_timed(x, w_gate, gate_bias, w1, w3, w2, top_k, capacity_factor, act, out, ws,
                   events):
-    """moe_forward recording 7 torch.cuda.Event objects at its stage boundaries."""
+    """moe_forward recording 7 torch.cuda.Event objects at its stage boundaries
+    (None entries are not recorded)."""
     for ev in events:
-        if ev.cuda_event == 0:      # torch creates the CUDA event on first record
+        if ev is not None and ev.cuda_event == 0:   # torch creates the CUDA event on first record
             ev.record()
-    handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    handles = (ctypes.c_void_p * len(events))(*[None if ev is None else ev.cuda_event
+                                                for ev in events])
     T, H = x.shape
     E = w_gate.shape[1]
     F = 8 if act == "identity" else w1.shape[2]
