@@ -135,9 +135,10 @@ def _overlapped_experts(steps, x_perm, offsets, recv_kept, w1, w3, w2, act, G, e
     docstring); fills y_back (rows in the order of x_perm)."""
     H = x_perm.shape[1]
     halves = [(0, el // 2), (el // 2, el)]
-    recv_in = []                       # per group: [G] received row counts per source
-    bufs = []
+    recv_in = []                       # per group: its counts [G, group size], row starts
+    bufs = []                          # per group: the received rows
     pending = []
+    keep = []                          # outputs still being sent back
     for gi, (j0, j1) in enumerate(halves):
         rk = recv_kept[:, j0:j1]
         cnt = rk.sum(axis=1)
@@ -168,8 +169,10 @@ def _overlapped_experts(steps, x_perm, offsets, recv_kept, w1, w3, w2, act, G, e
         recvs = [_rows(y_back, int(offsets[d * el + j0]), int(offsets[d * el + j1]))
                  for d in range(G)]
         back.append(_post(sends, recvs, me, group, tag=2 + gi))
+        keep.append(y_in)
     for w in back:
         _wait(w)
+    del keep
 
 
 def ep_forward(x, w_gate, gate_bias, w1_local, w3_local, w2_local, top_k: int,
