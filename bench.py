@@ -64,13 +64,23 @@ def parse_args(argv=None):
                     help="time plain device copies at the memory stages' sizes and exit")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds for the oracle baseline sample")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="token count T in place of the workload's (a sweep over batch x\n"
+                         "sequence length; the workload is then named <name>_T<T>)")
     return ap.parse_args(argv)
 
 
-def resolve_config(name: str) -> synth.MoEConfig:
+def resolve_config(name: str, tokens=None) -> synth.MoEConfig:
     if name.isdigit():
         name = synth.NUMBERED[int(name) - 1]
-    return synth.CONFIGS[name]
+    cfg = synth.CONFIGS[name]
+    if tokens is not None:
+        if tokens < 1:
+            raise ValueError("--tokens must be at least 1")
+        from dataclasses import replace
+        cfg = replace(cfg, T=int(tokens), name=f"{cfg.name}_T{int(tokens)}",
+                      description=f"{cfg.description}; T set to {int(tokens)} tokens")
+    return cfg
 
 
 def workload_desc(cfg: synth.MoEConfig) -> dict:
@@ -406,7 +416,7 @@ def run_op(args) -> int:
 
 def main(argv=None):
     args = parse_args(argv)
-    cfg = resolve_config(args.config)
+    cfg = resolve_config(args.config, args.tokens)
     if args.impl == "reference":
         return run_reference(args, cfg)
     if args.hbm_copy_sweep:
