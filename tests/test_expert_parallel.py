@@ -97,8 +97,10 @@ CASES = {
     "empty_rank": ((50, 0), 64, 64, 4, 2, "swiglu", "bf16", 1.25, None),
     "one_rank_gets_nothing": ((40, 40), 64, 64, 4, 2, "swiglu", "bf16", 0.0, "first_half"),
     "top1_many_experts": ((70, 33), 32, 64, 16, 1, "gelu", "f32", 1.0, None),
+    # four ranks
+    "four_ranks_drops": ((48, 0, 31, 64), 64, 128, 8, 2, "swiglu", "bf16", 0.75, None),
+    "four_ranks_top3": ((20, 45, 33, 7), 32, 64, 16, 3, "gelu", "f32", 0.0, None),
 }
-WORLD = 2
 
 
 def _free_port() -> int:
@@ -124,13 +126,13 @@ def _case_inputs(name, rank):
                 dtype=dtype, cf=cf)
 
 
-def _rank_main(rank: int, port: int, names, q):
+def _rank_main(rank: int, world: int, port: int, names, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         for name in names:
             d = _case_inputs(name, rank)
-            E, el = d["E"], d["E"] // WORLD
+            E, el = d["E"], d["E"] // world
             sl = slice(rank * el, (rank + 1) * el)
             local = lambda w: None if w is None else w[sl].contiguous()  # noqa: E731
             outs = [EP.ep_forward(d["x"], d["w_gate"], d["gate_bias"], local(d["w1"]),
@@ -154,14 +156,15 @@ def _rank_main(rank: int, port: int, names, q):
         dist.destroy_process_group()
 
 
-def test_expert_parallel_equals_single_device_forward_two_ranks():
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_equals_single_device_forward(world):
     ctx = mp.get_context("spawn")
     q = ctx.SimpleQueue()
-    names = sorted(CASES)
-    mp.start_processes(_rank_main, args=(_free_port(), names, q), nprocs=WORLD,
+    names = sorted(n for n in CASES if len(CASES[n][0]) == world)
+    mp.start_processes(_rank_main, args=(world, _free_port(), names, q), nprocs=world,
                        start_method="spawn", join=True)
-    res = [q.get() for _ in range(WORLD * len(names))]
-    assert len(res) == WORLD * len(names)
+    res = [q.get() for _ in range(world * len(names))]
+    assert len(res) == world * len(names)
     for name, rank, err, same in res:
         assert err <= TOL[CASES[name][6]], (name, rank, err)
         assert same >= 0.999, (name, rank, same)   # the same arithmetic row for row
