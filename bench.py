@@ -56,10 +56,13 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["layer", "expert_matmul", "route_stats"], default="layer",
+    ap.add_argument("--op", choices=["layer", "expert_matmul", "route_stats", "ep_one_rank"],
+                    default="layer",
                     help="layer: the MoE layer (default, the headline); expert_matmul: the k=1\n"
                          "up-projection op on x[1024,4096] x W[8,4096,14336]; route_stats: the\n"
-                         "router with its load statistics on the e32_long router shape")
+                         "router with its load statistics on the e32_long router shape;\n"
+                         "ep_one_rank: the expert-parallel forward on one NCCL rank (its\n"
+                         "exchanges and host reads) against the fused forward, --config workload")
     ap.add_argument("--hbm-copy-sweep", action="store_true",
                     help="time plain device copies at the memory stages' sizes and exit")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -346,6 +349,42 @@ def _time_steps(fn, steps: int, warmup: int, flush) -> list:
     return [a.elapsed_time(b) for a, b in ms]
 
 
+def _run_ep_one_rank(args, B, dev, flush, steps, warmup) -> int:
+    """The expert-parallel forward on a one-rank NCCL group: what its exchanges (here
+    local), host reads of the split sizes and regroup cost against the fused forward."""
+    import torch.distributed as tdist
+    from routing_grouped_expert_moe_b200 import expert_parallel as EP
+    cfg = resolve_config(args.config, args.tokens)
+    d = synth.make_inputs(cfg)
+    g = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+    ws = B.alloc_workspace(B.workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k, cfg.act,
+                                             cfg.torch_dtype), dev)
+    out = torch.empty(cfg.T, cfg.H, dtype=cfg.torch_dtype, device=dev)
+    args_l = (g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], cfg.top_k,
+              cfg.capacity_factor, cfg.act)
+    tdist.init_process_group("nccl", store=tdist.HashStore(), rank=0, world_size=1)
+    try:
+        fused = _time_steps(lambda: B.forward(*args_l, out=out, ws=ws), steps, warmup, flush)
+        ep = _time_steps(lambda: EP.ep_forward(*args_l, cfg.E), steps, warmup, flush)
+        ep_ov = _time_steps(lambda: EP.ep_forward(*args_l, cfg.E, overlap=True), steps, warmup,
+                            flush)
+    finally:
+        tdist.destroy_process_group()
+    f_ms, e_ms, o_ms = (statistics.mean(v) for v in (fused, ep, ep_ov))
+    line = {"metric": "expert-parallel layer tokens/s on one rank", "value": cfg.T / (e_ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+            "ms_per_step": e_ms, "higher_is_better": True, "dtype": cfg.dtype,
+            "data": "synthetic (seeded Philox normal inputs, random-init weights)",
+            "config": {**workload_desc(cfg), "l2": "flushed before every step",
+                       "parallelism": "ep1 (one NCCL rank: every exchange is a local copy)"},
+            "fused_forward_ms": f_ms, "ep_ms": e_ms, "ep_overlap_ms": o_ms,
+            "note": "CUDA events around each call on the current stream; the expert-parallel "
+                    "path reads its split sizes on the host twice per forward, and the GPU "
+                    "idles meanwhile"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_op(args) -> int:
     """One JSON line for a single-op row (not the layer headline)."""
     from routing_grouped_expert_moe_b200 import binding as B
@@ -354,6 +393,8 @@ def run_op(args) -> int:
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     peaks, peak_src = load_peaks()
     steps, warmup = min(args.steps, 100), max(args.warmup, 3)
+    if args.op == "ep_one_rank":
+        return _run_ep_one_rank(args, B, dev, flush, steps, warmup)
     if args.op == "expert_matmul":
         T, H, I, E, seed = 1024, 4096, 14336, 8, 5001
         x = synth.normal(seed, synth.STREAM_X, (T, H), 1.0, torch.bfloat16).to(dev)
