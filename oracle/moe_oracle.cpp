@@ -155,8 +155,7 @@ int oracle_topk_gates_literal(const float* logits, const int32_t* idx, int T, in
   return 0;
 }
 
-// Threshold gating: p = softmax over all E (the keep/drop decision in float32,
-// as the kernel takes it; NaN logits carry no mass);
+// Threshold gating: p = softmax over all E (float64, NaN logits carry no mass);
 // keep the experts with p > delta, largest first (ties to the lower id), at most
 // k_max, the largest always; g_s = exp(l_s - l_0) / sum_kept exp(l_j - l_0).
 // delta <= 0: 1/E (as float32).  idx/gate padded with -1 / 0.
@@ -173,15 +172,14 @@ int oracle_threshold_select(const float* logits, int T, int E, int k_max, float 
       while (pos > 0 && ranks_before(l[e], e, l[order[pos - 1]], order[pos - 1])) --pos;
       order.insert(order.begin() + pos, e);
     }
-    // the keep/drop decision in float32, the precision the kernel takes it in
-    float mx = -INFINITY;
+    double mx = -INFINITY;
     for (int e = 0; e < E; ++e)
-      if (!std::isnan(l[e])) mx = std::fmax(mx, l[e]);
-    float den = 0.0f;
+      if (!std::isnan(l[e])) mx = std::fmax(mx, static_cast<double>(l[e]));
+    double den = 0.0;
     for (int e = 0; e < E; ++e)
-      if (!std::isnan(l[e])) den += std::exp(l[e] - mx);
+      if (!std::isnan(l[e])) den += std::exp(static_cast<double>(l[e]) - mx);
     int n = 1;
-    while (n < k_max && std::exp(l[order[n]] - mx) / den > static_cast<float>(d)) ++n;
+    while (n < k_max && std::exp(static_cast<double>(l[order[n]]) - mx) / den > d) ++n;
     double z[64], zs = 0.0;
     for (int s = 0; s < n; ++s) {
       z[s] = std::exp(static_cast<double>(l[order[s]]) - static_cast<double>(l[order[0]]));

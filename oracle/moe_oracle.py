@@ -24,11 +24,21 @@ Sources (the pages this restates):
        ch.8: moe_router(x, router_weight, expert_weights, top_k,
        normalize_scores=True, capacity_factor=1.2).
 
-Readings where the pages are silent (each also listed with its reason in the
-design notes): capacity C = ceil(cf*T*k/E); overflow dropped first-come in
-token order; no second renormalisation after a drop; selection on fp32 logits,
-ties to the lower expert id, NaN below -inf; slot 0 = highest logit; exact erf
-GELU; SwiGLU = silu(x W1) * (x W3); h, y and out rounded to the storage dtype.
+Readings where the pages are silent:
+  * capacity C = ceil(cf*T*k/E) per expert per call, cf <= 0 meaning no limit
+    (the hnwysp.cn article names only an over-allocation coefficient);
+  * overflow dropped first come, first kept, in token order then slot order
+    (the workloads state "overflow dropped in token-index order");
+  * no second renormalisation after a drop: a dropped slot contributes nothing
+    and a token whose every slot dropped gives a zero row;
+  * selection on the fp32 logits (softmax is increasing, so the set and order
+    are those of the probabilities), ties to the lower expert id, NaN below
+    -inf, slot 0 = the largest logit;
+  * exact erf GELU, z * Phi(z); SwiGLU = silu(x W1) * (x W3), no expert biases;
+  * h, y and out rounded to the storage dtype (round to nearest even) where
+    the layer stores them;
+  * threshold gating keeps at most k_max experts, the largest always, and
+    decides p > delta on the float64 softmax.
 
 Arithmetic: every sum is float64.  Inputs arrive as float arrays holding the
 exact stored values (bf16 and fp32 values are exact in float64).  Rounding to
@@ -341,8 +351,7 @@ def combine(y, gates, row_map, dtype: str) -> np.ndarray:
 
 
 def threshold_select(logits, k_max: int, delta=None) -> dict:
-    """Per token: p = softmax over all E (the decision in float32, as the kernel
-    takes it); keep the experts with p > delta,
+    """Per token: p = softmax over all E (float64); keep the experts with p > delta,
     largest first (ties to the lower id), at most k_max; when none exceeds delta
     the largest alone is kept.  Gates g_s = exp(l_s - l_0) / sum_kept exp(l_j - l_0).
     delta None or <= 0: the default 1/E (as the float32 the library uses).
@@ -359,13 +368,11 @@ def threshold_select(logits, k_max: int, delta=None) -> dict:
         row = [float(v) for v in lg[t]]
         order = sorted(range(E), key=lambda e: (_rank_key(row[e]), e))
         l64 = np.asarray(row, dtype=np.float64)
-        # the keep/drop decision is taken in float32, the precision the kernel uses
-        l32 = lg[t].astype(np.float32)
-        z32 = np.exp(l32 - np.float32(np.nanmax(l32)), dtype=np.float32)
-        p32 = z32 / np.float32(np.nansum(z32, dtype=np.float32))
+        z = np.exp(l64 - np.nanmax(l64))
+        p = z / np.nansum(z)
         kept = [order[0]]
         for e in order[1:k_max]:
-            if not p32[e] > np.float32(d):
+            if not p[e] > d:
                 break
             kept.append(e)
         zk = np.exp(l64[kept] - l64[kept[0]])
