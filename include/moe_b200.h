@@ -13,7 +13,10 @@
  * ---------------------------------------
  * Ownership: the caller allocates and frees every buffer.  The library never
  *   allocates device memory; scratch comes from a caller-provided workspace
- *   `ws` of at least moe_workspace_bytes(...) bytes (256-byte aligned).
+ *   `ws` of at least moe_workspace_bytes(...) bytes (256-byte aligned).  The
+ *   one exception is moe_permute_noalloc: it takes no workspace, keeps its
+ *   scratch in library-owned device memory and reports kernel-found errors
+ *   only through its status_out argument.
  * Pointers: device pointers unless stated otherwise, 16-byte aligned.
  * Layouts: dense row-major.  x[T,H]; w_gate[H,E]; w1,w3[E,H,F]; w2[E,F,H];
  *   topk_idx / topk_gate / row_map [T,top_k]; x_perm, y [rows,H]; h [rows,F].
@@ -299,6 +302,47 @@ moe_status moe_selftest_epilogue_activations(const float* z, int n, float* gelu_
  * completion never arrives — and the kernel returns, leaving the context
  * usable.  Read the result with moe_get_device_status().                    */
 moe_status moe_selftest_bounded_wait(void* ws, moe_stream_t stream);
+
+/* Where the fused forward (moe_forward, moe_forward_timed,
+ * moe_forward_threshold) leaves its intermediates inside ws, for tests and
+ * tools that read them after the call has completed (no counterpart on the
+ * pages).  For the given sizes, writes the byte offset of section `which`
+ * from the start of ws and its size in bytes.  Contents once the forward has
+ * completed, valid until ws is reused:
+ *   MOE_WS_TOPK_IDX   int32 [T,k]   (only when topk_idx_out was NULL)
+ *   MOE_WS_TOPK_GATE  fp32  [T,k]
+ *   MOE_WS_COUNTS     int32 [E]     pre-drop (only when expert_counts_out was NULL)
+ *   MOE_WS_OFFSETS    int32 [E+1]   post-drop exclusive prefix, R = offsets[E]
+ *   MOE_WS_ROW_TOKEN  int32 [T*k]   first R entries written
+ *   MOE_WS_ROW_MAP    int32 [T,k]   -1 = dropped
+ *   MOE_WS_X_PERM     dt    [T*k,H] first R rows written (bf16 only)
+ *   MOE_WS_H          dt    [T*k,F] first R rows written
+ *   MOE_WS_Y          dt    [T*k,H] first R rows written
+ * Returns MOE_ERR_INVALID_ARG for bad sizes, enums or null outputs.          */
+typedef enum {
+  MOE_WS_TOPK_IDX = 0,
+  MOE_WS_TOPK_GATE = 1,
+  MOE_WS_COUNTS = 2,
+  MOE_WS_OFFSETS = 3,
+  MOE_WS_ROW_TOKEN = 4,
+  MOE_WS_ROW_MAP = 5,
+  MOE_WS_X_PERM = 6,
+  MOE_WS_H = 7,
+  MOE_WS_Y = 8
+} moe_ws_section;
+moe_status moe_workspace_section(int T, int H, int F, int E, int top_k, moe_act act,
+                                 moe_dtype dt, moe_ws_section which, size_t* offset,
+                                 size_t* bytes);
+
+/* Tuning hook (no counterpart on the pages): selects the bf16 grouped-GEMM
+ * kernel for the calls that follow, process-wide, so tests and benchmarks can
+ * run each one.  0 = automatic (the default, or MOE_GEMM_VARIANT read once
+ * when the library loads); 1 = row tiles of 128 rows, one CTA each; 2 = row
+ * tiles of 256 rows on CTA pairs; 3 = token-as-N tiles on CTA pairs (the
+ * tokens of an expert as the MMA's N; dense A rows only, gathered rows use
+ * the automatic choice).  Returns MOE_ERR_INVALID_ARG for other values.
+ * Not synchronised with calls running on other host threads.               */
+moe_status moe_set_gemm_variant(int variant);
 
 /* Synchronises `stream`, then returns the status the kernels of the last
  * call(s) on this workspace recorded (MOE_OK when none), and clears it.      */

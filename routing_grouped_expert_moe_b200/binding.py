@@ -61,6 +61,8 @@ _SIGS = {
                                    _p, _p, _p, _sz, _p]),
     "moe_selftest_epilogue_activations": (_i, [_p, _i, _p, _p, _p]),
     "moe_selftest_bounded_wait": (_i, [_p, _p]),
+    "moe_workspace_section": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p]),
+    "moe_set_gemm_variant": (_i, [_i]),
     "moe_get_device_status": (_i, [_p, _p]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
@@ -500,3 +502,25 @@ def selftest_bounded_wait(ws):
 def device_status(ws) -> int:
     """Synchronises the current stream and returns (and clears) the kernels' status word."""
     return int(_lib.moe_get_device_status(_ptr(ws), _stream()))
+
+
+WS_SECTIONS = {"topk_idx": 0, "topk_gate": 1, "counts": 2, "offsets": 3, "row_token": 4,
+               "row_map": 5, "x_perm": 6, "h": 7, "y": 8}
+GEMM_VARIANTS = {"auto": 0, "rows128": 1, "rows256_pair": 2, "tokens_pair": 3}
+
+
+def workspace_section(ws, name, T, H, F, E, top_k, act="swiglu", dtype=torch.bfloat16):
+    """The view of section `name` of a fused-forward workspace (uint8 tensor
+    `ws`), per moe_workspace_section: read it once the forward has completed."""
+    off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(_lib.moe_workspace_section(T, H, F, E, top_k, ACT[act], BF16 if dtype == torch.bfloat16 else F32,
+                                      WS_SECTIONS[name], ctypes.byref(off), ctypes.byref(nb)),
+           "moe_workspace_section")
+    return ws[off.value:off.value + nb.value]
+
+
+def set_gemm_variant(variant) -> None:
+    """Select the bf16 grouped-GEMM kernel process-wide ("auto", "rows128",
+    "rows256_pair", "tokens_pair", or 0..3), per moe_set_gemm_variant."""
+    v = GEMM_VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    _check(_lib.moe_set_gemm_variant(v), "moe_set_gemm_variant")

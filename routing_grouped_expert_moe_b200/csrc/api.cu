@@ -2,6 +2,7 @@
 // workspace layout and the launch sequence of each entry point.  No entry
 // point allocates device memory or synchronises the stream (except
 // moe_get_device_status, whose job is to synchronise).
+#include <atomic>
 #include <climits>
 #include <cstdlib>
 #include <cmath>
@@ -14,10 +15,31 @@
 using namespace moe;
 
 namespace moe {
-bool pdl_enabled() {
-  const char* e = getenv("MOE_PDL");
-  return !(e && e[0] == '0');
+namespace {
+int env_int(const char* name, int dflt) {
+  const char* e = getenv(name);
+  return (e && e[0]) ? atoi(e) : dflt;
 }
+Tuning read_tuning() {
+  Tuning t;
+  t.pdl = env_int("MOE_PDL", 1) != 0;
+  const int v = env_int("MOE_GEMM_VARIANT", 0);
+  t.gemm_variant = (v >= 1 && v <= 3) ? v : 0;
+  t.gemm_ctas = env_int("MOE_GEMM_CTAS", 0);
+  t.epi_sleep_ns = env_int("MOE_EPI_SLEEP", t.epi_sleep_ns);
+  if (t.epi_sleep_ns < 0) t.epi_sleep_ns = 0;
+  t.route_split_cap = env_int("MOE_ROUTE_SPLIT", 0);
+  t.route_shallow = env_int("MOE_ROUTE_DEEP", 1) == 0;
+  t.tokn_nacc = env_int("MOE_TOKN_NACC", 0);
+  t.tokn_bk = env_int("MOE_TOKN_BK", 0);
+  return t;
+}
+// Initialised when the library is loaded.
+const Tuning g_tuning = read_tuning();
+std::atomic<int> g_gemm_variant{g_tuning.gemm_variant};
+}  // namespace
+const Tuning& tuning() { return g_tuning; }
+int gemm_variant() { return g_gemm_variant.load(std::memory_order_relaxed); }
 }  // namespace moe
 
 namespace {
@@ -43,12 +65,19 @@ int num_sms_current() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace: [status | topk_idx | topk_gate | tile_counts | tickets | partials |
+// Workspace: [status | topk_idx | topk_gate | tile_counts | sched + tickets | partials |
 //             counts | offsets | row_token | row_map | x_perm | h | y | x_stage | out_stage]
+// sched: the grouped GEMMs' tile counters (kSchedCounters ints), directly
+// followed by the router's tickets, so one clear covers both.
+constexpr int kSchedCounters = 4;
 struct WsLayout {
-  size_t status, topk_idx, topk_gate, tile_counts, tickets, partials, counts, offsets, row_token,
-      row_map, x_perm, h, y, x_stage, out_stage, logits, n_sel, total;
+  size_t status, topk_idx, topk_gate, tile_counts, sched, tickets, partials, counts, offsets,
+      row_token, row_map, x_perm, h, y, x_stage, out_stage, logits, n_sel, total;
 };
+
+// Workspaces that begin with the status word's 256-byte block keep the GEMMs'
+// tile counters in that block, 16 bytes in.
+constexpr size_t kSchedInStatusBlock = 16;
 
 WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt, bool host_stage,
                    bool threshold = false) {
@@ -61,7 +90,9 @@ WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt,
   L.topk_idx = o;    o = align_up(o + R * 4);
   L.topk_gate = o;   o = align_up(o + R * 4);
   L.tile_counts = o; o = align_up(o + tiles * E * 4);
-  L.tickets = o;     o = align_up(o + (static_cast<size_t>(T) / 128 + 1) * 4);
+  L.sched = o;
+  L.tickets = o + kSchedCounters * 4;
+  o = align_up(L.tickets + (static_cast<size_t>(T) / 128 + 1) * 4);
   L.partials = o;    o = align_up(o + static_cast<size_t>(kRouteMaxCtas) * 128 * E * 4);
   L.counts = o;      o = align_up(o + static_cast<size_t>(E) * 4);
   L.offsets = o;     o = align_up(o + static_cast<size_t>(E + 1) * 4);
@@ -112,10 +143,11 @@ int capacity_of(float cf, int T, int k, int E) {
 cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // Grouped FFN on prepared buffers (shared by moe_grouped_ffn and moe_forward).
+// sched: two zeroed tile counters (GEMM-1, GEMM-2).
 moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, const void* w1,
                    const void* w3, const void* w2, const int32_t* offsets, int R_max, int T,
                    int H, int F, int E, moe_act act, moe_dtype dt, void* y, void* h, int* status,
-                   cudaStream_t s, cudaEvent_t mid_event = nullptr) {
+                   int* sched, cudaStream_t s, cudaEvent_t mid_event = nullptr) {
   const int nsm = num_sms_current();
   const bool gather = row_token != nullptr;
   const void* a_src = gather ? x : x_perm;
@@ -140,6 +172,7 @@ moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, 
   g.N = F;
   g.K = H;
   g.out = h;
+  g.sched = sched;
   cudaError_t err;
   if (dt == MOE_BF16)
     err = launch_gemm_tc(mode1, gather, a_src, a_rows, w1, w3, g, nsm, s);
@@ -152,6 +185,7 @@ moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, 
   g.N = H;
   g.K = F;
   g.out = y;
+  g.sched = sched + 1;
   if (dt == MOE_BF16)
     err = launch_gemm_tc(2, false, h, R_max, w2, nullptr, g, nsm, s);
   else
@@ -273,9 +307,10 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
   if (ws_bytes < h_off) return MOE_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
   int* status = at<int>(ws, 0);
-  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  int* sched = at<int>(ws, kSchedInStatusBlock);
+  if (launch_clear_status(status, s, sched, 2) != cudaSuccess) return MOE_ERR_CUDA;
   return run_ffn(x_perm, row_token, x, w1, w3, w2, expert_offsets, R_max, T, H, F, E, act, dt, y,
-                 at<void>(ws, h_off), status, s);
+                 at<void>(ws, h_off), status, sched, s);
 }
 
 moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
@@ -391,7 +426,8 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
   int* status = at<int>(ws, 0);
-  if (launch_clear_status(status, s) != cudaSuccess) return MOE_ERR_CUDA;
+  int* sched = at<int>(ws, kSchedInStatusBlock);
+  if (launch_clear_status(status, s, sched, 1) != cudaSuccess) return MOE_ERR_CUDA;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* row_map = at<int32_t>(ws, L.row_map);
   void* x_perm = at<void>(ws, L.x_perm);
@@ -416,7 +452,7 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
   GemmArgs g{};
   g.offsets = offsets;
   g.E = E; g.R_max = T; g.T = T; g.status = status;
-  g.N = I; g.K = H; g.out = y;
+  g.N = I; g.K = H; g.out = y; g.sched = sched;
   const cudaError_t err =
       dt == MOE_BF16 ? launch_gemm_tc(2, false, x_perm, T, expert_weight, nullptr, g,
                                       num_sms_current(), s)
@@ -493,8 +529,10 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   void* x_perm = bf16 ? at<void>(ws, L.x_perm) : nullptr;
 
   auto mark = [&](int i) { return ev && ev[i] ? cudaEventRecord(ev[i], s) : cudaSuccess; };
+  int* sched = at<int>(ws, L.sched);
   int* tickets = at<int>(ws, L.tickets);
-  if (launch_clear_status(status, s, tickets, T / 128 + 1) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_clear_status(status, s, sched, kSchedCounters + T / 128 + 1) != cudaSuccess)
+    return MOE_ERR_CUDA;
   // 1. route (+ per-tile histogram)
   if (mark(0) != cudaSuccess) return MOE_ERR_CUDA;
   RouteArgs ra{};
@@ -545,7 +583,7 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   const int R_max = T * top_k;
   void* y = at<void>(ws, L.y);
   st = run_ffn(x_perm, bf16 ? nullptr : row_token, x, w1, w3, w2, offsets, R_max, T, H, F, E, act,
-               dt, y, at<void>(ws, L.h), status, s, ev ? ev[4] : nullptr);
+               dt, y, at<void>(ws, L.h), status, sched, s, ev ? ev[4] : nullptr);
   if (st != MOE_OK) return st;
   if (mark(5) != cudaSuccess) return MOE_ERR_CUDA;
   // 4. combine
@@ -728,6 +766,38 @@ moe_status moe_forward_host_batches(const void* const* x_host, void* const* out_
     st = st == MOE_OK ? MOE_ERR_CUDA : st;
   for (int i = 0; i < 7; ++i) cudaEventDestroy(ev[i]);  // released once their work completes
   return st;
+}
+
+moe_status moe_workspace_section(int T, int H, int F, int E, int top_k, moe_act act,
+                                 moe_dtype dt, moe_ws_section which, size_t* offset,
+                                 size_t* bytes) {
+  if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU && act != MOE_ACT_IDENTITY)
+    return MOE_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0 || F <= 0 || E <= 0 || top_k <= 0 || !offset || !bytes)
+    return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(T, H, F, E, top_k, act, dt, false);
+  const size_t R = static_cast<size_t>(T) * top_k;
+  const size_t eb = elem_bytes(dt);
+  switch (which) {
+    case MOE_WS_TOPK_IDX: *offset = L.topk_idx; *bytes = R * 4; break;
+    case MOE_WS_TOPK_GATE: *offset = L.topk_gate; *bytes = R * 4; break;
+    case MOE_WS_COUNTS: *offset = L.counts; *bytes = static_cast<size_t>(E) * 4; break;
+    case MOE_WS_OFFSETS: *offset = L.offsets; *bytes = static_cast<size_t>(E + 1) * 4; break;
+    case MOE_WS_ROW_TOKEN: *offset = L.row_token; *bytes = R * 4; break;
+    case MOE_WS_ROW_MAP: *offset = L.row_map; *bytes = R * 4; break;
+    case MOE_WS_X_PERM: *offset = L.x_perm; *bytes = R * H * eb; break;
+    case MOE_WS_H: *offset = L.h; *bytes = act == MOE_ACT_IDENTITY ? 0 : R * F * eb; break;
+    case MOE_WS_Y: *offset = L.y; *bytes = R * H * eb; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_set_gemm_variant(int variant) {
+  if (variant < 0 || variant > 3) return MOE_ERR_INVALID_ARG;
+  moe::g_gemm_variant.store(variant, std::memory_order_relaxed);
+  return MOE_OK;
 }
 
 moe_status moe_get_device_status(void* ws, moe_stream_t stream) {

@@ -21,10 +21,6 @@ constexpr int G_EPI_WARPS = 8;
 constexpr int G_STG_BYTES = 32 * 32 * 2;  // one epilogue warp's staging box: 32 rows x 32 bf16
 constexpr int G_SMEM = G_STAGES * G_STAGE_BYTES + G_EPI_WARPS * G_STG_BYTES + 1024;
 constexpr uint32_t G_TMEM_COLS = 512;
-// Default L2 prefetch distance of the GEMM producers, in k-blocks (0: off).
-constexpr int kGemmPrefetchDist = 0;
-// Default sleep of an epilogue warp between polls of its accumulator barrier.
-constexpr int kEpilogueSleepNs = 1000;
 
 template <int MODE>
 struct ModeCfg {
@@ -315,13 +311,14 @@ inline bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D bf16 map over W[E, K, N] (N contiguous), box {64 N, 64 K, 1}, 128-byte swizzle.
-inline bool make_map_w(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
+// 3-D bf16 map over W[E, K, N] (N contiguous), box {64 N, box_k K, 1}, 128-byte swizzle.
+inline bool make_map_w(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N,
+                       uint32_t box_k = 64) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {N, K, E};
   cuuint64_t strides[2] = {N * 2, K * N * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, box_k, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

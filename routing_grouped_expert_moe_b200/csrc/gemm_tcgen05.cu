@@ -27,7 +27,6 @@
 // quarter split the tile's columns, so the activation epilogue of one tile
 // finishes within the next tile's main loop).
 #include <cmath>
-#include <cstdlib>
 
 #include "gemm_common.cuh"
 
@@ -131,34 +130,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           r4[j] = i < ti.rows ? args.row_token[ti.m0 + i] : first;
         }
       }
-      // L2 prefetch runs pf_dist k-blocks ahead of the ring, into the CTA's
-      // next tile once this one is covered.
-      const bool has_next = tau + static_cast<int>(gridDim.x) < total;
-      const TileInfo nx = has_next ? decode_tile(tau + gridDim.x, s_prefix, s_seg_start, s_seg_rows,
-                                                 s_mtiles, E, BN_OUT)
-                                   : ti;
-      auto prefetch_kb = [&](const TileInfo& t, int k0) {
-        if (!GATHER) tma_prefetch_l2_2d(&tmA, k0, t.m0);
-        if (MODE == 1) {
-          tma_prefetch_l2_3d(&tmB1, t.n0, k0, t.e);
-          tma_prefetch_l2_3d(&tmB1, t.n0 + 64, k0, t.e);
-          tma_prefetch_l2_3d(&tmB3, t.n0, k0, t.e);
-          tma_prefetch_l2_3d(&tmB3, t.n0 + 64, k0, t.e);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) tma_prefetch_l2_3d(&tmB1, t.n0 + 64 * j, k0, t.e);
-        }
-      };
       bool ok = true;
       for (int kb = 0; kb < num_kb; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, args.status);
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        if (lane == 0 && args.pf_dist > 0) {
-          const int j = kb + args.pf_dist;
-          if (j < num_kb) prefetch_kb(ti, j * G_BK);
-          else if (has_next && j - num_kb < num_kb) prefetch_kb(nx, (j - num_kb) * G_BK);
-        }
         uint8_t* sA = smem + stage * G_STAGE_BYTES;
         uint8_t* sB = sA + G_A_BYTES;
         const int k0 = kb * G_BK;
@@ -298,21 +274,19 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const 
   return launch_kernel(kern, dim3(num_sms), dim3(G_THREADS), G_SMEM, s, 1, a, b1, b3, o, g);
 }
 
-// Kernel variant: one CTA per 128-row tile, or CTA pairs sharing 256-row
-// tiles (gemm_tcgen05_pair.cu).  Pairs cut each SM's operand traffic per
-// k-block from 48 KB to 32 KB, which makes a pair tile ~8% faster than a
-// one-CTA tile of the same rows (measured 0.92-0.94), but round every expert
-// up to 256 rows and run on half as many tile slots.  The host does not know
-// the expert counts (they stay on the device), so it compares the expected
-// number of waves for balanced experts of a = R_max / E rows: an expert of
-// about a rows takes a / BM + 1/2 row tiles on average (its count straddles a
-// tile boundary).  MOE_GEMM_VARIANT=1|2 forces one.
-static int forced_variant() {
-  const char* e = getenv("MOE_GEMM_VARIANT");
-  return (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
-}
-
-static int choose_variant(int mode, const GemmArgs& g, int num_sms) {
+// Kernel variant for dense A rows: the token-as-N pair kernel (gemm_tokn.cu:
+// weights as the MMA's M, an expert's tokens as N, rounded up to 16 instead of
+// to a 128- or 256-row tile, and fewer operand bytes per MMA clock), or the
+// row-tiled kernels, one CTA per 128-row tile (1) or CTA pairs sharing 256-row
+// tiles (2).  Gathered A rows (row_token) use the row-tiled kernels: the pair
+// when the expected wave count for balanced experts of a = R_max / E rows
+// (a / BM + 1/2 row tiles per expert; a pair tile counted at 0.92 of a one-CTA
+// tile, as measured) is lower.  The tuning variant forces one.
+static int choose_variant(int mode, bool gather, const GemmArgs& g, int num_sms) {
+  const int forced = gemm_variant();
+  if (forced == 3 && !gather) return 3;
+  if (forced == 1 || forced == 2) return forced;
+  if (!gather) return 3;
   const double a = static_cast<double>(g.R_max) / g.E;
   const double n_tiles = std::ceil(static_cast<double>(g.N) / (mode == 1 ? 128 : 256));
   const double t1 = g.E * (a / G_BM + 0.5) * n_tiles;
@@ -324,6 +298,14 @@ static int choose_variant(int mode, const GemmArgs& g, int num_sms) {
 
 cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
                            const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s) {
+  GemmArgs ga = g;
+  ga.epi_sleep_ns = tuning().epi_sleep_ns;
+  // a cap on the persistent grid (measurement aid: how the GEMM scales with SMs)
+  const int cap = tuning().gemm_ctas;
+  if (cap >= 2 && cap < num_sms) num_sms = cap;
+  const int variant = choose_variant(mode, gather, g, num_sms);
+  if (variant == 3 && g.sched != nullptr)
+    return launch_gemm_tokn(mode, a_src, a_rows, b1, b3, ga, num_sms, s);
   CUtensorMap ma, mb1, mb3, mo;
   // A: [a_rows, K]; dense source uses 128-row boxes, the gathered source 1-row boxes.
   if (!make_map_2d(&ma, a_src, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(g.K),
@@ -337,21 +319,6 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
   }
   if (!make_map_out(&mo, g.out, static_cast<uint64_t>(g.R_max), static_cast<uint64_t>(g.N)))
     return cudaErrorInvalidValue;
-  // MOE_GEMM_PF=<k-blocks> sets the L2 prefetch distance (0 turns it off).
-  GemmArgs ga = g;
-  ga.pf_dist = kGemmPrefetchDist;
-  if (const char* e = getenv("MOE_GEMM_PF")) ga.pf_dist = atoi(e) < 0 ? 0 : atoi(e);
-  // MOE_EPI_SLEEP=<ns> sets the epilogue warps' sleep between accumulator polls.
-  ga.epi_sleep_ns = kEpilogueSleepNs;
-  if (const char* e = getenv("MOE_EPI_SLEEP")) ga.epi_sleep_ns = atoi(e) < 0 ? 0 : atoi(e);
-  // MOE_GEMM_CTAS=<n> caps the persistent grid (a measurement aid: how the
-  // GEMM scales with the number of SMs it runs on).
-  if (const char* e = getenv("MOE_GEMM_CTAS")) {
-    const int n = atoi(e);
-    if (n >= 2 && n < num_sms) num_sms = n;
-  }
-  int variant = forced_variant();
-  if (variant == 0) variant = choose_variant(mode, g, num_sms);
   if (variant == 2) return launch_gemm_tc_pair(mode, gather, ma, mb1, mb3, mo, ga, num_sms, s);
   switch (mode * 2 + (gather ? 1 : 0)) {
     case 0: return launch_tc<0, false>(ma, mb1, mb3, mo, ga, num_sms, s);

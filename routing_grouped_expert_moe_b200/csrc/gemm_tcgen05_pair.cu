@@ -153,34 +153,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           r4[j] = i < ti.rows ? args.row_token[ti.m0 + i] : first;
         }
       }
-      // L2 prefetch of this CTA's own boxes, pf_dist k-blocks ahead of the
-      // ring, running into the pair's next tile once this one is covered.
-      const bool has_next = tau + npairs < total;
-      const PairTile nx = has_next ? decode_pair(tau + npairs, s_prefix, s_seg_start, s_seg_rows,
-                                                 s_mtiles, E, BN_OUT, static_cast<int>(rank))
-                                   : ti;
-      auto prefetch_kb = [&](const PairTile& t, int k0) {
-        if (!GATHER && t.rows > 0) tma_prefetch_l2_2d(&tmA, k0, t.m0);
-        if (MODE == 1) {
-          const CUtensorMap* mb = rank == 0 ? &tmB1 : &tmB3;
-          tma_prefetch_l2_3d(mb, t.n0, k0, t.e);
-          tma_prefetch_l2_3d(mb, t.n0 + 64, k0, t.e);
-        } else {
-          const int nb = t.n0 + 128 * static_cast<int>(rank);
-          tma_prefetch_l2_3d(&tmB1, nb, k0, t.e);
-          tma_prefetch_l2_3d(&tmB1, nb + 64, k0, t.e);
-        }
-      };
       bool ok = true;
       for (int kb = 0; kb < num_kb; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, args.status);
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        if (lane == 0 && args.pf_dist > 0) {
-          const int j = kb + args.pf_dist;
-          if (j < num_kb) prefetch_kb(ti, j * G_BK);
-          else if (has_next && j - num_kb < num_kb) prefetch_kb(nx, (j - num_kb) * G_BK);
-        }
         uint8_t* sA = smem + stage * P_STAGE_BYTES;
         uint8_t* sB = sA + P_A_BYTES;
         const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);

@@ -10,13 +10,31 @@ namespace moe {
 constexpr int kMaxE = 256;
 constexpr int kMaxTopK = 8;
 
+// ---------------------------------------------------------------- tuning
+// Measurement aids, read from the environment once when the library is loaded
+// (never on a launch path).  The defaults are the product configuration.
+struct Tuning {
+  bool pdl = true;              // MOE_PDL=0: launch without programmatic dependent launch
+  int gemm_variant = 0;         // MOE_GEMM_VARIANT=1|2|3: the initial grouped-GEMM choice
+  int gemm_ctas = 0;            // MOE_GEMM_CTAS=n: cap the persistent GEMM grid at n CTAs
+  int epi_sleep_ns = 1000;      // MOE_EPI_SLEEP=ns: epilogue warps' sleep between polls
+  int route_split_cap = 0;      // MOE_ROUTE_SPLIT=1..16: cap the router's split of H
+  bool route_shallow = false;   // MOE_ROUTE_DEEP=0: keep the router's shallow ring
+  int tokn_nacc = 0;            // MOE_TOKN_NACC=1|2: accumulators per tile of the GELU/down GEMMs
+  int tokn_bk = 0;              // MOE_TOKN_BK=64|128: K per pipeline stage of the token-as-N GEMM
+};
+const Tuning& tuning();
+// Grouped-GEMM kernel choice: 0 automatic, 1 | 2 | 3 forced (moe_set_gemm_variant;
+// starts as Tuning::gemm_variant).
+int gemm_variant();
+
 // ---------------------------------------------------------------- launches
 // Programmatic dependent launch: with it on, a kernel's CTAs may be scheduled
 // while its predecessor in the stream is finishing, and run their prologue;
 // every kernel of this library executes griddepcontrol.wait (pdl_wait) before
 // it touches global memory, which returns once the predecessor grid has
-// completed and its writes are visible.  MOE_PDL=0 turns the attribute off.
-bool pdl_enabled();
+// completed and its writes are visible.
+inline bool pdl_enabled() { return tuning().pdl; }
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -108,17 +126,16 @@ struct GemmArgs {
   int T;                     // rows of the gathered source
   void* out;                 // [R_max, N]
   int* status;
-  int pf_dist;               // k-blocks ahead of the TMA ring to prefetch into L2 (0: off)
+  int* sched;                // tile counter of the dynamic schedule (zero before the launch)
   int epi_sleep_ns;          // epilogue warps' sleep between polls of the accumulator barrier
-};
-
-struct GemmTcPlan {
-  CUtensorMap tmA, tmB1, tmB3;
 };
 
 // bf16 tensor-core (tcgen05) path. a_src: x_perm/h rows (dense) or x (gather).
 cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
                            const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s);
+// Token-as-N variant on CTA pairs (dense A rows only; needs g.sched).
+cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void* b1,
+                             const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s);
 // CTA-pair variant (cta_group::2), tensor maps prepared by launch_gemm_tc.
 cudaError_t launch_gemm_tc_pair(int mode, bool gather, const CUtensorMap& ma,
                                 const CUtensorMap& mb1, const CUtensorMap& mb3,

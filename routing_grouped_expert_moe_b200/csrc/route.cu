@@ -191,11 +191,9 @@ RoutePlan route_plan(int T, int H, int E, int dt_bf16, int num_sms, bool can_spl
     while (p.ck < 16 && p.tiles * p.ck * 2 <= kRouteMaxCtas && p.tiles * p.ck * 2 <= num_sms &&
            num_kb >= 4 * p.ck)
       p.ck *= 2;
-  // MOE_ROUTE_SPLIT=1|2|4|8|16 caps the split (measurement aid)
-  if (const char* env = getenv("MOE_ROUTE_SPLIT")) {
-    const int cap = atoi(env);
-    while (cap >= 1 && p.ck > cap) p.ck >>= 1;
-  }
+  // a cap on the split (measurement aid)
+  const int cap = tuning().route_split_cap;
+  while (cap >= 1 && p.ck > cap) p.ck >>= 1;
   return p;
 }
 

@@ -316,11 +316,6 @@ static int num_sms_for_route() {
   return n;
 }
 
-// MOE_ROUTE_DEEP=0 keeps the shallow ring (a measurement aid).
-static bool route_shallow_forced() {
-  const char* e = getenv("MOE_ROUTE_DEEP");
-  return e && e[0] == '0';
-}
 
 // W_gate [H, E] as a 2-D map (E contiguous), 64 x 64 boxes, 128-byte swizzle;
 // experts beyond E read as zeros.
@@ -349,7 +344,7 @@ static cudaError_t launch_route_tc_nkd(const CUtensorMap& mx, const CUtensorMap&
 template <int NPAD, int K>
 static cudaError_t launch_route_tc_nk(const CUtensorMap& mx, const CUtensorMap& mw,
                                       const RouteArgs& a, int tiles, int S, cudaStream_t s) {
-  if (tiles * S <= num_sms_for_route() && !route_shallow_forced())
+  if (tiles * S <= num_sms_for_route() && !tuning().route_shallow)
     return launch_route_tc_nkd<NPAD, K, true>(mx, mw, a, tiles, S, s);
   return launch_route_tc_nkd<NPAD, K, false>(mx, mw, a, tiles, S, s);
 }

@@ -25,3 +25,19 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture
+def gemm_variant():
+    """Selects the bf16 grouped-GEMM kernel for one test (moe_set_gemm_variant)
+    and restores the automatic choice afterwards."""
+    from routing_grouped_expert_moe_b200 import binding
+    chosen = []
+
+    def set_variant(v):
+        binding.set_gemm_variant(v)
+        chosen.append(v)
+
+    yield set_variant
+    if chosen:
+        binding.set_gemm_variant(0)

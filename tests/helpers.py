@@ -85,3 +85,70 @@ def rel_err(gpu, ref) -> float:
     if denom == 0.0:
         return float(np.max(np.abs(g))) if g.size else 0.0
     return float(np.max(np.abs(g - r)) / denom)
+
+
+# ---------------------------------------------------------------- canary guards
+# compute-sanitizer is not available on the GPU pool, so device buffers handed to
+# the library are surrounded by sentinel bytes; a kernel that writes past an
+# output (or into a part of the workspace it must not touch) changes them.
+CANARY = 0xA5
+MARGIN = 4096  # bytes before and after every guarded buffer
+
+
+class Guarded:
+    """A device tensor of `shape`/`dtype` inside a uint8 allocation whose MARGIN
+    bytes on either side (and, optionally, the tensor itself) hold CANARY."""
+
+    def __init__(self, shape, dtype, device="cuda", fill_canary=True):
+        n = 1
+        for s in shape:
+            n *= int(s)
+        self.nbytes = n * torch.empty(0, dtype=dtype).element_size()
+        self.raw = torch.full((self.nbytes + 2 * MARGIN,), CANARY, dtype=torch.uint8,
+                              device=device)
+        self.bytes = self.raw[MARGIN:MARGIN + self.nbytes]
+        self.t = self.bytes.view(dtype).view(*shape)
+        if not fill_canary:
+            self.t.zero_()
+
+    def check(self, what="buffer"):
+        torch.cuda.synchronize()
+        lo = self.raw[:MARGIN]
+        hi = self.raw[MARGIN + self.nbytes:]
+        bad_lo = int((lo != CANARY).sum())
+        bad_hi = int((hi != CANARY).sum())
+        assert bad_lo == 0 and bad_hi == 0, \
+            f"{what}: {bad_lo} bytes changed before it, {bad_hi} after it"
+
+    def untouched(self, start_byte, end_byte, what="region"):
+        """Asserts bytes [start, end) of the tensor still hold CANARY."""
+        torch.cuda.synchronize()
+        seg = self.bytes[start_byte:end_byte]
+        bad = int((seg != CANARY).sum())
+        assert bad == 0, f"{what}: {bad} of {end_byte - start_byte} bytes written"
+
+
+def guarded_workspace(nbytes, device="cuda") -> Guarded:
+    """A 256-byte-aligned workspace (MARGIN is a multiple of 256) filled with CANARY."""
+    return Guarded((int(nbytes),), torch.uint8, device)
+
+
+def check_forward_workspace(ws: Guarded, B, cfg, R: int, act=None, what=""):
+    """After a fused forward: the workspace's margins are intact, and the rows
+    past the R kept rows of x_perm, h and y, and the row_token entries past R,
+    were never written (the permute writes R rows, the GEMMs write only rows of
+    their experts' segments)."""
+    act = act or cfg.act
+    ws.check(f"{what} workspace")
+    T, k = cfg.T, cfg.top_k
+    eb = 2 if cfg.dtype == "bf16" else 4
+    for name, width, esize in (("row_token", 1, 4), ("x_perm", cfg.H, eb), ("h", cfg.F, eb),
+                               ("y", cfg.H, eb)):
+        if name == "x_perm" and cfg.dtype != "bf16":
+            continue
+        if name == "h" and act == "identity":
+            continue
+        sec = B.workspace_section(ws.t, name, T, cfg.H, cfg.F, cfg.E, k, act, cfg.torch_dtype)
+        off = sec.data_ptr() - ws.t.data_ptr()
+        ws.untouched(off + R * width * esize, off + T * k * width * esize,
+                     f"{what} {name} past row {R}")

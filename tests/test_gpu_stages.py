@@ -10,7 +10,7 @@ import torch
 
 from oracle import moe_oracle as O
 from routing_grouped_expert_moe_b200 import synth
-from tests.helpers import TOL, as_np, gap_violations, rel_err
+from tests.helpers import Guarded, guarded_workspace, TOL, as_np, gap_violations, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -149,27 +149,45 @@ def _ffn_case(dtype, act, E, rows_per_expert, H, F, seed=11):
     (2, [300, 45], 512, 1376),             # F of the 32-expert workload (N tail 1376 % 256)
     (5, [512, 640, 383, 0, 129], 384, 512),   # even / odd m-tile counts per expert
 ])
-@pytest.mark.parametrize("variant", ["1", "2"], ids=["cta1", "cta2"])
-def test_grouped_ffn(dtype, act, gather, shape, variant, monkeypatch):
-    if dtype == "f32" and variant == "2":
+@pytest.mark.parametrize("variant", ["rows128", "rows256_pair", "tokens_pair"])
+def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
+    """Every kernel against the oracle, with R_max - R = 37 spare rows: the spare
+    rows of x_perm hold NaN (a kernel that mixes rows would spread them), the
+    spare rows of y and the bytes around y and the workspace hold sentinels
+    that must survive."""
+    if dtype == "f32" and variant != "rows128":
         pytest.skip("the fp32 path has a single CUDA-core kernel")
-    monkeypatch.setenv("MOE_GEMM_VARIANT", variant)
+    if gather and variant == "tokens_pair":
+        pytest.skip("gathered rows always use the row-tiled kernels")
+    gemm_variant(variant)
     E, rows, H, F = shape
     dt, x, w1, w3, w2, perm = _ffn_case(dtype, act, E, rows, H, F)
     xo = as_np(x)
     ref = O.grouped_ffn(xo, perm, as_np(w1), None if w3 is None else as_np(w3), as_np(w2), act,
                         dtype, E)
+    R = perm["R"]
+    R_max = R + 37
     offs = torch.from_numpy(perm["offsets"].astype(np.int32)).cuda()
-    rt = torch.from_numpy(perm["row_token"].astype(np.int32)).cuda()
+    rt = torch.full((R_max,), 0, dtype=torch.int32)
+    rt[:R] = torch.from_numpy(perm["row_token"].astype(np.int32))
+    esz = 2 if dtype == "bf16" else 4
+    y = Guarded((R_max, H), dt)
+    ws = guarded_workspace(256 + R_max * F * esz)
     if gather:
-        y = B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
-                            x=x.cuda(), row_token=rt)
+        B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
+                        x=x.cuda(), row_token=rt.cuda(), R_max=R_max, ws=ws.t, y=y.t)
     else:
-        x_perm = x[torch.from_numpy(perm["row_token"])].contiguous().cuda()
-        y = B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
-                            x_perm=x_perm)
+        x_perm = torch.full((R_max, H), float("nan"), dtype=dt)
+        x_perm[:R] = x[torch.from_numpy(perm["row_token"])]
+        B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
+                        x_perm=x_perm.cuda(), R_max=R_max, ws=ws.t, y=y.t)
     torch.cuda.synchronize()
-    assert rel_err(as_np(y)[:perm["R"]], ref) <= TOL[dtype]
+    got = as_np(y.t)[:R]
+    assert np.all(np.isfinite(got))
+    assert rel_err(got, ref) <= TOL[dtype]
+    y.check("y")
+    y.untouched(R * H * esz, R_max * H * esz, "y rows past R")
+    ws.check("workspace")
 
 
 def test_grouped_ffn_identity_and_gemm_only_rows():
