@@ -58,6 +58,18 @@ struct TokCfg {
   static_assert(STAGES >= 2, "pipeline needs two stages");
 };
 
+// Token rows one CTA loads per 64-wide K chunk for half_n needed rows
+// (8 <= half_n <= 128, a multiple of 8): a first box of 32, 64 or 128 rows and,
+// for 65-96 rows, a second box of 32 rows placed after it.
+struct TokRows {
+  int first, second;
+};
+__host__ __device__ constexpr TokRows tok_rows(int half_n) {
+  return half_n <= 32 ? TokRows{32, 0}
+                      : (half_n <= 64 ? TokRows{64, 0}
+                                      : (half_n <= 96 ? TokRows{64, 32} : TokRows{128, 0}));
+}
+
 struct TokTile {
   int e, row0, rows, n, col0;
 };
@@ -300,9 +312,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                                       C::COLS_PER_TILE);
         const int half_n = ti.n >> 1;
         // this CTA's token rows: one box of 32, 64 or 128 rows, or 64 + 32
-        const int rows_ld = (half_n + 31) & ~31;
-        const CUtensorMap* xa = rows_ld <= 32 ? &tmX32 : (rows_ld <= 64 ? &tmX64 : &tmX128);
-        const bool x_second = rows_ld == 96;  // a 32-row box after a 64-row one
+        const TokRows xr = tok_rows(half_n);
+        const int rows_ld = xr.first + xr.second;
+        const CUtensorMap* xa = xr.first == 32 ? &tmX32 : (xr.first == 64 ? &tmX64 : &tmX128);
+        const bool x_second = xr.second != 0;  // a 32-row box after a 64-row one
         const int xrow = ti.row0 + static_cast<int>(rank) * half_n;
         const uint32_t tx = 2u * static_cast<uint32_t>(C::A_BYTES + (BK / 64) * rows_ld * 128);
         const int wcol = ti.col0 + 128 * static_cast<int>(rank);
@@ -478,7 +491,17 @@ static cudaError_t launch_tokn_bk(int bk, const CUtensorMap* x, const CUtensorMa
 cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void* b1,
                              const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s) {
   if (g.sched == nullptr) return cudaErrorInvalidValue;
-  const int bk = tuning().tokn_bk == 64 ? 64 : 128;
+  // Tile shape per GEMM (measured on the Mixtral-shaped and page-1 layers):
+  // SwiGLU keeps two accumulators (W1, W3) and 4 stages of K = 64; GELU one
+  // double-buffered accumulator and 3 stages of K = 128; the down-projection
+  // likewise, unless its token rows (R_max x K) outgrow half of L2, where two
+  // accumulators per token tile halve their re-reads (4 stages of K = 64).
+  bool two = mode == 1;
+  if (mode == 2)
+    two = static_cast<double>(g.R_max) * g.K * 2.0 > 64.0 * 1024 * 1024;
+  int bk = two ? 64 : 128;
+  if (mode != 1 && tuning().tokn_nacc != 0) two = tuning().tokn_nacc == 2;
+  if (tuning().tokn_bk != 0) bk = tuning().tokn_bk == 64 ? 64 : 128;
   CUtensorMap mx[3], mw1, mw3, mo;
   const uint32_t box_rows[3] = {32, 64, 128};
   for (int i = 0; i < 3; ++i)
@@ -494,7 +517,6 @@ cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void
   }
   if (!make_map_out(&mo, g.out, static_cast<uint64_t>(g.R_max), static_cast<uint64_t>(g.N)))
     return cudaErrorInvalidValue;
-  const bool two = tuning().tokn_nacc != 1;
   switch (mode) {
     case 0: return two ? launch_tokn_bk<0, 2>(bk, mx, mw1, mw3, mo, g, num_sms, s)
                        : launch_tokn_bk<0, 1>(bk, mx, mw1, mw3, mo, g, num_sms, s);

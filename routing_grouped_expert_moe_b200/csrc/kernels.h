@@ -20,8 +20,8 @@ struct Tuning {
   int epi_sleep_ns = 1000;      // MOE_EPI_SLEEP=ns: epilogue warps' sleep between polls
   int route_split_cap = 0;      // MOE_ROUTE_SPLIT=1..16: cap the router's split of H
   bool route_shallow = false;   // MOE_ROUTE_DEEP=0: keep the router's shallow ring
-  int tokn_nacc = 0;            // MOE_TOKN_NACC=1|2: accumulators per tile of the GELU/down GEMMs
-  int tokn_bk = 0;              // MOE_TOKN_BK=64|128: K per pipeline stage of the token-as-N GEMM
+  int tokn_nacc = 0;            // MOE_TOKN_NACC=1|2: force the accumulators per tile (GELU, down)
+  int tokn_bk = 0;              // MOE_TOKN_BK=64|128: force the K per pipeline stage
 };
 const Tuning& tuning();
 // Grouped-GEMM kernel choice: 0 automatic, 1 | 2 | 3 forced (moe_set_gemm_variant;
