@@ -56,6 +56,15 @@ struct TokCfg {
   static constexpr int COLS_PER_TILE = MODE == 1 ? 256 : 256 * NACC;  // output columns per tile
   static constexpr int SMEM = STAGES * STAGE_BYTES + G_EPI_WARPS * NBOX * G_STG_BYTES + 1024;
   static_assert(STAGES >= 2, "pipeline needs two stages");
+  // TMA producer warps.  One issuing thread streams at about half the rate an
+  // SM can take (measured: 31 B/clk with one warp, 60 with two, 64 with four,
+  // same boxes and stages), so PROD warps (warp 0, then warps 10, 11, ...)
+  // each own the stages s = p mod PROD.  PROD divides STAGES: a stage always
+  // has the same producer, which never gets more than one lap ahead of the
+  // MMA on it (the empty barrier's parity tells only one lap from the next).
+  static constexpr int PROD = STAGES <= 4 ? STAGES : (STAGES % 3 == 0 ? 3 : 2);
+  static_assert(STAGES % PROD == 0, "every stage needs a single producer");
+  static constexpr int THREADS = G_THREADS + 32 * (PROD - 1);
 };
 
 // Token rows one CTA loads per 64-wide K chunk for half_n needed rows
@@ -158,7 +167,7 @@ __device__ __forceinline__ void tok_activate(float (&v)[32], const float (&u)[32
 }  // namespace
 
 template <int MODE, int NACC, int BK>
-__global__ void __launch_bounds__(G_THREADS, 1)
+__global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
     k_gemm_tokn(const __grid_constant__ CUtensorMap tmX32, const __grid_constant__ CUtensorMap tmX64,
                 const __grid_constant__ CUtensorMap tmX128, const __grid_constant__ CUtensorMap tmW1,
                 const __grid_constant__ CUtensorMap tmW3, const __grid_constant__ CUtensorMap tmO,
@@ -202,7 +211,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
     for (int i = 0; i < T_SD; ++i) {
       mbar_init(&sched_full[i], 1);
-      mbar_init(&sched_empty[i], G_EPI_WARPS + (rank == 0 ? 1 : 0));
+      // consumers: the epilogue warps, the other producers, the MMA warp (first CTA)
+      mbar_init(&sched_empty[i], G_EPI_WARPS + (C::PROD - 1) + (rank == 0 ? 1 : 0));
       mbar_init(&mb_full[i], 1);
       mbar_init(&mb_empty[i], 1);
     }
@@ -281,16 +291,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     return __shfl_sync(0xffffffffu, tau, 0);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ tile fetch + TMA producer
+  if (warp == 0 || warp >= 2 + G_EPI_WARPS) {
+    // ------------------------------------------------------------ tile fetch + TMA producers
+    // Producer p issues the stages whose running index g (over all tiles and
+    // k-blocks) is p mod PROD, i.e. ring stages p, p + PROD, ...; producer 0
+    // also fetches the tiles.
+    const int p = warp == 0 ? 0 : warp - (1 + G_EPI_WARPS);
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      uint32_t g = 0;
       for (int i = 0;; ++i) {
         const int slot = i % T_SD;
         const uint32_t ph = static_cast<uint32_t>(i / T_SD) & 1u;
         int tau;
-        if (rank == 0) {
+        if (p != 0) {
+          if (!mbar_wait(&sched_full[slot], ph, abort_flag, args.status)) break;
+          tau = vs_tile[slot];
+          mbar_arrive(&sched_empty[slot]);
+        } else if (rank == 0) {
           if (!mbar_wait(&sched_empty[slot], ph ^ 1u, abort_flag, args.status)) break;
           if (!mbar_wait(&mb_empty[slot], ph ^ 1u, abort_flag, args.status)) break;
           tau = atomicAdd(args.sched, 1);
@@ -320,7 +337,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const uint32_t tx = 2u * static_cast<uint32_t>(C::A_BYTES + (BK / 64) * rows_ld * 128);
         const int wcol = ti.col0 + 128 * static_cast<int>(rank);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          if (g % C::PROD != static_cast<uint32_t>(p)) continue;
+          const int stage = static_cast<int>(g % C::STAGES);
+          const uint32_t phase = (g / C::STAGES) & 1u;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, args.status)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sX = sA + C::A_BYTES;
@@ -346,7 +366,6 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             if (x_second)
               tma_load_2d_pair(sX + c * T_XCHUNK + 64 * 128, &tmX32, bar, k0 + 64 * c, xrow + 64);
           }
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
       }
@@ -476,7 +495,7 @@ static cudaError_t launch_tokn_t(const CUtensorMap* x, const CUtensorMap& w1,
   auto kern = k_gemm_tokn<MODE, NACC, BK>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
-  return launch_kernel(kern, dim3((num_sms / 2) * 2), dim3(G_THREADS), C::SMEM, s, 2, x[0], x[1],
+  return launch_kernel(kern, dim3((num_sms / 2) * 2), dim3(C::THREADS), C::SMEM, s, 2, x[0], x[1],
                        x[2], w1, w3, o, g);
 }
 
