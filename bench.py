@@ -333,6 +333,55 @@ def hbm_copy_sweep() -> int:
     return 0
 
 
+def copy_us(nbytes: int, flush, dev, reps: int = 10) -> float:
+    """Median CUDA-event microseconds of one plain device copy that moves nbytes in
+    all (nbytes/2 read, nbytes/2 written), L2 flushed before each copy."""
+    n = max(1, nbytes // 4)
+    a = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    ts = []
+    for i in range(reps + 3):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        b.copy_(a)
+        s1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(s0.elapsed_time(s1) * 1000.0)
+    return statistics.median(ts)
+
+
+def kernels_per_call(fn) -> int | None:
+    """Kernel launches one call of fn makes, counted as the kernel nodes of a CUDA
+    graph captured from it (None when the graph cannot be inspected)."""
+    try:
+        from cuda.bindings import runtime as rt
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        graph = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        count = 0
+        for node in nodes[:n]:
+            err, typ = rt.cudaGraphNodeGetType(node)
+            if typ == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                count += 1
+        del g
+        torch.cuda.synchronize()
+        return count
+    except Exception as e:  # pragma: no cover - inspection is best effort
+        print(f"kernels_per_call: {e!r}", file=sys.stderr)
+        return None
+
+
 def _time_steps(fn, steps: int, warmup: int, flush) -> list:
     """CUDA-event milliseconds of each of `steps` calls (L2 flushed before each)."""
     for _ in range(warmup):
@@ -538,7 +587,6 @@ def main(argv=None):
     total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(T, world, args.steps, total_ms)
-    gpu_launches = 6 * args.steps   # clear-status, route, scatter (+scan), GEMM-1, GEMM-2, combine
 
     # the timed steps in three parts: status clear + route + scatter, the two expert
     # GEMMs, the combine
@@ -558,6 +606,16 @@ def main(argv=None):
     names = ["route", "scan", "scatter", "gemm1", "gemm2", "combine"]
     stage_ms = {n: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_stage))
                 for j, n in enumerate(names)}
+
+    # ---- the library's kernel launches per forward (kernel nodes of a captured graph)
+    per_fwd = kernels_per_call(fwd)
+    gpu_launches = (per_fwd if per_fwd is not None else 6) * args.steps
+
+    # ---- a plain device copy of each memory stage's algorithmic bytes (the rate
+    # the stage could reach at its size: launch and ramp dominate small copies)
+    same_copy_us = {"route": copy_us(work["route_bytes"], flush, dev),
+                    "scatter": copy_us(work["scatter_bytes"], flush, dev),
+                    "combine": copy_us(work["combine_bytes"], flush, dev)}
 
     # ---- end to end through the host-buffer entry point (H2D + layer + D2H)
     n_e2e = min(args.steps, 50)
@@ -648,6 +706,8 @@ def main(argv=None):
                            "mode": "one call per step: copy-in, layer, copy-out in turn on one "
                                    "stream, L2 flushed before each step"}},
         "gpu_launches": gpu_launches,
+        "gpu_launches_source": ("kernel nodes of one captured forward x steps" if per_fwd
+                                is not None else "plan: 6 kernels per forward x steps"),
         "roofline": {"kernel": "k_gemm_tokn (expert GEMM-1 + GEMM-2)", "bound": "tensor",
                      "achieved": gemm_tflops, "peak": tc, "unit": "TFLOP/s",
                      "frac": gemm_tflops / tc, "peak_source": f"{peak_src} burst bf16",
@@ -667,6 +727,11 @@ def main(argv=None):
                           "route_gbs_detail": work["route_bytes"] / (stage_ms["route"] / 1e3)
                           / 1e9},
         "combine": {"gbs": comb_gbs, "frac_measured_hbm": comb_gbs / hbm},
+        "memory_stages_vs_same_size_copy": {
+            n: {"stage_us": 1000.0 * stage_ms[n], "copy_us": same_copy_us[n],
+                "bytes": work[f"{n}_bytes"],
+                "frac_of_same_size_copy": same_copy_us[n] / (1000.0 * stage_ms[n])}
+            for n in ("route", "scatter", "combine")},
         "timed_parts_us": {n: 1000.0 * v for n, v in part_ms.items()},
         "stage_us_detail": {n: 1000.0 * v for n, v in stage_ms.items()},
         "stage_detail": f"every kernel apart: {n_stage} forwards with events at all stage "

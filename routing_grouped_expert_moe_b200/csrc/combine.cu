@@ -7,8 +7,9 @@
 // article §2.2, stage 3); here each token reads its own k rows and sums them in
 // slot order, so the result is the same bit for bit on every run.
 //
-// One warp per token, 16-byte vector loads of each kept row, fp32 accumulation
-// by FMA in slot order, one rounding to the storage type.  A null gate array
+// One warp per token (or per part of a token's row when there are few tokens),
+// 16-byte vector loads of each kept row, fp32 accumulation by FMA in slot
+// order, one rounding to the storage type.  A null gate array
 // means every weight is 1 (the unpermute of a k = 1 matmul: out[t] = y[row]).
 #include "common.cuh"
 #include "kernels.h"
@@ -60,17 +61,24 @@ __device__ __forceinline__ void combine_store(const int4 (&q)[kMaxTopK],
   *reinterpret_cast<int4*>(dst) = o;
 }
 
+// Work item w (one warp): token w / split, and every split-th chunk of 64
+// vectors of its row starting at chunk w % split (split > 1 when there are too
+// few tokens to fill the GPU with warps).
 template <bool BF16>
 __global__ void __launch_bounds__(kCombineThreads)
     k_combine(const uint8_t* __restrict__ y, const float* __restrict__ gate,
-              const int32_t* __restrict__ row_map, int T, int H, int k, uint8_t* __restrict__ out) {
+              const int32_t* __restrict__ row_map, int T, int H, int k, int split,
+              uint8_t* __restrict__ out) {
   pdl_wait_and_trigger();
   constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
   constexpr int EB = BF16 ? 2 : 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nvec = H / EPV;
-  for (int t = blockIdx.x * (kCombineThreads / 32) + warp; t < T;
-       t += gridDim.x * (kCombineThreads / 32)) {
+  const long long items = static_cast<long long>(T) * split;
+  for (long long w = static_cast<long long>(blockIdx.x) * (kCombineThreads / 32) + warp;
+       w < items; w += static_cast<long long>(gridDim.x) * (kCombineThreads / 32)) {
+    const int t = static_cast<int>(w / split);
+    const int part = static_cast<int>(w % split);
     int rows[kMaxTopK];
     float g[kMaxTopK];
 #pragma unroll
@@ -80,7 +88,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
     // two 16-byte vectors per lane and round: every load of both is in flight
     // before the first FMA
-    for (int v0 = lane; v0 < nvec; v0 += 64) {
+    for (int v0 = part * 64 + lane; v0 < nvec; v0 += 64 * split) {
       const int v1 = v0 + 32;
       const bool two = v1 < nvec;
       int4 qa[kMaxTopK], qb[kMaxTopK];
@@ -106,16 +114,23 @@ __global__ void __launch_bounds__(kCombineThreads)
 cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
                            int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s) {
   const int warps_per_cta = kCombineThreads / 32;
-  int grid = (T + warps_per_cta - 1) / warps_per_cta;
-  const int cap = num_sms * 8;  // resident CTAs; larger T loops inside the kernel
+  // split a row over several warps when the tokens alone leave the GPU short
+  // of warps (about 32 per SM keep enough loads in flight)
+  const int chunks = (H / (dt_bf16 ? 8 : 4) + 63) / 64;
+  int split = (num_sms * 32) / (T > 0 ? T : 1);
+  if (split > chunks) split = chunks;
+  if (split < 1) split = 1;
+  const long long items = static_cast<long long>(T) * split;
+  long long grid = (items + warps_per_cta - 1) / warps_per_cta;
+  const long long cap = static_cast<long long>(num_sms) * 8;  // resident CTAs; more loop inside
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   if (dt_bf16)
-    return launch_kernel(k_combine<true>, dim3(grid), dim3(kCombineThreads), 0, s, 1,
-                         static_cast<const uint8_t*>(y), gate, row_map, T, H, k,
+    return launch_kernel(k_combine<true>, dim3(static_cast<unsigned>(grid)), dim3(kCombineThreads),
+                         0, s, 1, static_cast<const uint8_t*>(y), gate, row_map, T, H, k, split,
                          static_cast<uint8_t*>(out));
-  return launch_kernel(k_combine<false>, dim3(grid), dim3(kCombineThreads), 0, s, 1,
-                       static_cast<const uint8_t*>(y), gate, row_map, T, H, k,
+  return launch_kernel(k_combine<false>, dim3(static_cast<unsigned>(grid)), dim3(kCombineThreads),
+                       0, s, 1, static_cast<const uint8_t*>(y), gate, row_map, T, H, k, split,
                        static_cast<uint8_t*>(out));
 }
 

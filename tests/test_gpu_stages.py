@@ -46,6 +46,9 @@ def test_route_from_logits_bit_exact(T, E, k):
     ("bf16", 300, 256, 256, 8),                     # 256 experts (MMA N = 256), top-8
     ("bf16", 19000, 192, 128, 2),                   # 128 experts, no H split, ragged tail
     ("bf16", 50, 64, 12, 3),                        # E not a multiple of 8 (CUDA-core path)
+    ("bf16", 777, 2048, 16, 2),                     # few experts: H split in a cluster, ragged tile
+    ("bf16", 129, 768, 8, 3),                       # few experts, one CTA per tile
+    ("bf16", 4096, 256, 16, 1),                     # few experts, top-1
     ("f32", 257, 128, 4, 2), ("f32", 100, 96, 40, 3),
 ])
 def test_route_from_x(dtype, T, H, E, k):
