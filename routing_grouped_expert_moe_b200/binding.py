@@ -171,8 +171,9 @@ def route_from_logits(logits, top_k):
     return idx, gate
 
 
-def permute(token_expert_idx, num_experts, capacity_factor=0.0, x=None, ws=None):
-    """Dispatch: returns dict(counts, offsets, row_token, row_map[, x_perm])."""
+def permute(token_expert_idx, num_experts, capacity_factor=0.0, x=None, ws=None, out=None):
+    """Dispatch: returns dict(counts, offsets, row_token, row_map[, x_perm]).
+    out: optional dict of preallocated output tensors under those names."""
     _need(token_expert_idx, "token_expert_idx", dtype=torch.int32, dim=2)
     T, k = token_expert_idx.shape
     dev = token_expert_idx.device
@@ -182,11 +183,19 @@ def permute(token_expert_idx, num_experts, capacity_factor=0.0, x=None, ws=None)
         H, dt = x.shape[1], _dt(x)
     else:
         H, dt = 8, BF16
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    row_token = torch.full((T * k,), -1, dtype=torch.int32, device=dev)
-    row_map = torch.empty(T, k, dtype=torch.int32, device=dev)
-    x_perm = torch.empty(T * k, H, dtype=x.dtype, device=dev) if x is not None else None
+    out = out or {}
+    counts = out.get("counts", torch.empty(E, dtype=torch.int32, device=dev))
+    offsets = out.get("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    row_token = out.get("row_token", torch.full((T * k,), -1, dtype=torch.int32, device=dev))
+    row_map = out.get("row_map", torch.empty(T, k, dtype=torch.int32, device=dev))
+    x_perm = None
+    if x is not None:
+        x_perm = out.get("x_perm", torch.empty(T * k, H, dtype=x.dtype, device=dev))
+    for name, t, n in (("counts", counts, E), ("offsets", offsets, E + 1),
+                       ("row_token", row_token, T * k), ("row_map", row_map, T * k)):
+        _need(t, name, dtype=torch.int32)
+        if t.numel() != n or not t.is_contiguous():
+            raise ValueError(f"{name}: {n} contiguous int32 entries expected")
     if ws is None:
         ws = alloc_workspace(workspace_bytes(T, H, 8, E, k, "identity",
                                              torch.bfloat16 if dt == BF16 else torch.float32), dev)

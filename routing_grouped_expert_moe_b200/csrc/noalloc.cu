@@ -24,7 +24,13 @@
 //
 // The device address of the array is looked up once per device, with that
 // device current, by the first call on it (cudaGetSymbolAddress); make that
-// first call before any stream capture.
+// first call before any stream capture.  The address belongs to the device's
+// current context: a call that finds another context current (after
+// cudaDeviceReset, or once the primary context was released and created
+// again) looks it up again, so make the first call after such a reset before
+// any stream capture too.
+#include <cuda.h>
+
 #include <cmath>
 #include <mutex>
 
@@ -43,10 +49,30 @@ static __device__ __align__(256) int g_permute_scratch[kScratchInts];
 
 constexpr int kMaxDevices = 64;
 
-// Device address of g_permute_scratch on the current device (set-up on first use).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The context current on this thread (driver entry point; null if unavailable).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_permute_scratch on the current device, looked up on the
+// first call with the device's current context (and again if that context
+// changed since).
 int* scratch_on_current_device(cudaError_t* err) {
   static std::mutex mu;
   static int* addr[kMaxDevices] = {};
+  static CUcontext ctx_of[kMaxDevices] = {};
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return nullptr;
@@ -55,11 +81,13 @@ int* scratch_on_current_device(cudaError_t* err) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const CUcontext ctx = current_context();
+  if (addr[dev] == nullptr || ctx != ctx_of[dev]) {
     void* p = nullptr;
     *err = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (*err != cudaSuccess) return nullptr;
     addr[dev] = static_cast<int*>(p);
+    ctx_of[dev] = current_context();  // the runtime call made the primary context current
   }
   return addr[dev];
 }
@@ -106,7 +134,17 @@ extern "C" moe_status moe_permute_noalloc(const void* x, const int32_t* token_ex
   p.E = E;
   p.BT = kPermuteBT;
   p.tiles = tiles;
+  // as moe_permute: enough CTAs per tile to spread the x_perm copies (only the
+  // grid changes; the scratch holds one histogram row per tile either way)
   p.split = 1;
+  if (x_perm) {
+    int nsm = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      nsm = 148;
+    while (p.split < 16 && tiles * p.split < 2 * nsm) p.split *= 2;
+  }
   if (capacity_factor > 0.f) {  // C = ceil(cf * T * k / E), at least 1
     const double c =
         std::ceil(static_cast<double>(capacity_factor) * static_cast<double>(T) * top_k / E);

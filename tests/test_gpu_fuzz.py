@@ -8,7 +8,8 @@ import torch
 
 from oracle import moe_oracle as O
 from routing_grouped_expert_moe_b200 import synth
-from tests.helpers import TOL, as_np, gapped_inputs, rel_err
+from tests.helpers import (TOL, Guarded, as_np, check_forward_workspace, gapped_inputs,
+                           guarded_workspace, rel_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,17 +38,25 @@ CASES = _cases()
 
 @pytest.mark.parametrize("cfg", CASES, ids=lambda c: f"{c.name}-T{c.T}-H{c.H}-F{c.F}-E{c.E}-k{c.top_k}"
                                                       f"-{c.act}-{c.dtype}-cf{c.capacity_factor}")
-def test_forward_fuzz(cfg):
+def test_forward_fuzz(cfg, gemm_variant):
+    """Each case on one of the three bf16 GEMM kernels in turn; outputs and the
+    workspace sentinel-guarded, rows past R untouched."""
     from routing_grouped_expert_moe_b200 import binding as B
+    gemm_variant(["tokens_pair", "rows128", "rows256_pair"][int(cfg.name[4:]) % 3])
     d = gapped_inputs(cfg)
     g = {k: (None if v is None else v.cuda()) for k, v in d.items()}
-    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device="cuda")
-    cnt = torch.empty(cfg.E, dtype=torch.int32, device="cuda")
-    ws = B.alloc_workspace(B.workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k, cfg.act,
-                                             cfg.torch_dtype))
+    ig = Guarded((cfg.T, cfg.top_k), torch.int32)
+    cg = Guarded((cfg.E,), torch.int32)
+    og = Guarded((cfg.T, cfg.H), cfg.torch_dtype)
+    wsg = guarded_workspace(B.workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k, cfg.act,
+                                              cfg.torch_dtype))
+    idx, cnt = ig.t, cg.t
     out = B.forward(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], cfg.top_k,
-                    cfg.capacity_factor, cfg.act, ws=ws, topk_idx_out=idx, expert_counts_out=cnt)
-    assert B.device_status(ws) == B.OK
+                    cfg.capacity_factor, cfg.act, out=og.t, ws=wsg.t, topk_idx_out=idx,
+                    expert_counts_out=cnt)
+    assert B.device_status(wsg.t) == B.OK
+    for buf, name in ((ig, "topk_idx"), (cg, "counts"), (og, "out")):
+        buf.check(name)
     f = lambda t: None if t is None else as_np(t)  # noqa: E731
     ref = O.moe_forward(f(d["x"]), f(d["w_gate"]), f(d["gate_bias"]), f(d["w1"]), f(d["w3"]),
                         f(d["w2"]), cfg.top_k, cfg.capacity_factor, cfg.act, cfg.dtype)
@@ -55,6 +64,7 @@ def test_forward_fuzz(cfg):
     np.testing.assert_array_equal(as_np(cnt), ref["counts"])
     err = rel_err(as_np(out), ref["out"])
     assert err <= TOL[cfg.dtype], err
+    check_forward_workspace(wsg, B, cfg, int(ref["R"]), what=cfg.name)
 
 
 def _thr_cases(n=12, seed=778):

@@ -11,7 +11,7 @@ import torch
 from oracle import moe_oracle as O
 from oracle import moe_oracle_cpp as OC
 from routing_grouped_expert_moe_b200 import synth
-from tests.helpers import TOL, as_np, gapped_inputs, rel_err
+from tests.helpers import TOL, Guarded, as_np, gapped_inputs, guarded_workspace, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -38,8 +38,10 @@ def test_route_stats(cfg):
     d = gapped_inputs(cfg, with_weights=False)
     x, wg = d["x"].cuda(), d["w_gate"].cuda()
     b = None if d["gate_bias"] is None else d["gate_bias"].cuda()
-    idx, gate, counts, prob, ws = B().route_stats(x, wg, b, cfg.top_k)
+    wsg = guarded_workspace(B()._lib.moe_route_stats_workspace_bytes(cfg.T, cfg.E))
+    idx, gate, counts, prob, ws = B().route_stats(x, wg, b, cfg.top_k, ws=wsg.t)
     assert B().device_status(ws) == B().OK
+    wsg.check("workspace")
     # selection equals the oracle's (the inputs keep a 1e-3 gap between ranks)
     lg_ref = O.router_logits(as_np(d["x"]), as_np(d["w_gate"]),
                              None if d["gate_bias"] is None else as_np(d["gate_bias"]))
@@ -79,8 +81,13 @@ def _matmul_inputs(T, H, I, E, dtype, e_used, seed):
 def test_expert_matmul_full_compare(case):
     T, H, I, E, dtype, e_used = case
     x, w, ids = _matmul_inputs(T, H, I, E, dtype, e_used, seed=4000 + T)
-    out, ws = B().expert_matmul(x.cuda(), w.cuda(), ids.cuda())
+    og = Guarded((T, I), x.dtype)
+    wsg = guarded_workspace(B()._lib.moe_expert_matmul_workspace_bytes(T, H, I, E,
+                                                                       B()._dt(x)))
+    out, ws = B().expert_matmul(x.cuda(), w.cuda(), ids.cuda(), out=og.t, ws=wsg.t)
     assert B().device_status(ws) == B().OK
+    og.check("out")
+    wsg.check("workspace")
     for orc in (O, OC):
         ref = orc.expert_matmul(as_np(x), as_np(w), ids.numpy(), dtype)
         err = rel_err(as_np(out), ref)
@@ -152,11 +159,18 @@ def test_forward_threshold(cfg, k_max, cf):
     delta = float(np.float32(1.0 / cfg.E))
     d = threshold_inputs(cfg, delta, k_max)
     g = {k: (None if v is None else v.cuda()) for k, v in d.items()}
-    idx = torch.empty(cfg.T, k_max, dtype=torch.int32, device="cuda")
-    n = torch.empty(cfg.T, dtype=torch.int32, device="cuda")
+    ig = Guarded((cfg.T, k_max), torch.int32)
+    ng = Guarded((cfg.T,), torch.int32)
+    og = Guarded((cfg.T, cfg.H), cfg.torch_dtype)
+    wsg = guarded_workspace(B()._lib.moe_forward_threshold_workspace_bytes(
+        cfg.T, cfg.H, cfg.F, cfg.E, k_max, B().ACT[cfg.act], B()._dt(d["x"])))
+    idx, n = ig.t, ng.t
     out, ws = B().forward_threshold(g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"],
-                                    k_max, 0.0, cf, cfg.act, topk_idx_out=idx, n_selected_out=n)
+                                    k_max, 0.0, cf, cfg.act, out=og.t, ws=wsg.t,
+                                    topk_idx_out=idx, n_selected_out=n)
     assert B().device_status(ws) == B().OK
+    for buf, name in ((ig, "topk_idx"), (ng, "n_selected"), (og, "out"), (wsg, "workspace")):
+        buf.check(name)
     f = lambda t: None if t is None else as_np(t)  # noqa: E731
     for orc in (O, OC):
         ref = orc.moe_forward_threshold(f(d["x"]), f(d["w_gate"]), f(d["gate_bias"]), f(d["w1"]),

@@ -73,8 +73,20 @@ def test_route_from_x(dtype, T, H, E, k):
 # ---------------------------------------------------------------- permute
 
 def _perm_check(ids, E, cf, x=None):
-    r = B().permute(ids.cuda(), E, capacity_factor=cf, x=None if x is None else x.cuda())
-    cap = O.capacity(cf, ids.shape[0], ids.shape[1], E)
+    """moe_permute against the oracle bit for bit, every output and the
+    workspace sentinel-guarded; row_token entries and x_perm rows past R must
+    stay unwritten."""
+    T, k = ids.shape
+    H = 8 if x is None else x.shape[1]
+    g = {"counts": Guarded((E,), torch.int32), "offsets": Guarded((E + 1,), torch.int32),
+         "row_token": Guarded((T * k,), torch.int32), "row_map": Guarded((T, k), torch.int32)}
+    if x is not None:
+        g["x_perm"] = Guarded((T * k, H), x.dtype)
+    ws = guarded_workspace(B().workspace_bytes(T, H, 8, E, k, "identity",
+                                               torch.bfloat16 if x is None else x.dtype))
+    r = B().permute(ids.cuda(), E, capacity_factor=cf, x=None if x is None else x.cuda(),
+                    ws=ws.t, out={n: v.t for n, v in g.items()})
+    cap = O.capacity(cf, T, k, E)
     ref = O.permute(ids.numpy(), E, cap)
     np.testing.assert_array_equal(as_np(r["counts"]), ref["counts"])
     np.testing.assert_array_equal(as_np(r["offsets"]), ref["offsets"])
@@ -84,6 +96,12 @@ def _perm_check(ids, E, cf, x=None):
     assert B().device_status(r["ws"]) == B().OK
     if x is not None:
         np.testing.assert_array_equal(as_np(r["x_perm"])[:R], as_np(x)[ref["row_token"]])
+        g["x_perm"].untouched(R * H * x.element_size(), T * k * H * x.element_size(),
+                              "x_perm rows past R")
+    g["row_token"].untouched(R * 4, T * k * 4, "row_token past R")
+    for n, v in g.items():
+        v.check(n)
+    ws.check("workspace")
     return r, ref
 
 
@@ -213,9 +231,12 @@ def test_combine(dtype, T, H, k):
     row_map = rng.permutation(R).reshape(T, k).astype(np.int32)
     row_map[rng.random((T, k)) < 0.1] = -1          # some dropped slots
     gate = torch.from_numpy(rng.random((T, k)).astype(np.float32))
-    out = B().unpermute_combine(y.cuda(), gate.cuda(), torch.from_numpy(row_map).cuda())
+    og = Guarded((T, H), dt)
+    out = B().unpermute_combine(y.cuda(), gate.cuda(), torch.from_numpy(row_map).cuda(),
+                                out=og.t)
     ref = O.combine(as_np(y), gate.numpy(), row_map, dtype)
     assert rel_err(as_np(out), ref) <= (1e-6 if dtype == "f32" else 8e-3)
+    og.check("out")
     # deterministic: a second run is bit-identical
     out2 = B().unpermute_combine(y.cuda(), gate.cuda(), torch.from_numpy(row_map).cuda())
     assert torch.equal(out, out2)

@@ -79,3 +79,28 @@ def test_noalloc_permute_reports_bad_ids_and_rejects_oversize():
     st = B._lib.moe_permute_noalloc(None, p, big_T, 8, 256, 2, ctypes.c_float(0.0), B.BF16,
                                     None, p, p, p, p, None, None)
     assert st == B.ERR_UNSUPPORTED
+
+
+def test_noalloc_python_wrapper_matches_permute():
+    """binding.permute_noalloc (argument order, output allocation, the x = None
+    form and status_out) gives exactly what binding.permute gives."""
+    B = _lib()
+    T, E, k, cf = 999, 16, 2, 1.0
+    ids = synth.random_expert_ids(21, T, E, k, skew=0.2).cuda()
+    x = synth.normal(21, 0, (T, 128), 1.0, torch.bfloat16).cuda()
+    for with_x in (True, False):
+        for with_status in (True, False):
+            status = torch.full((1,), 99, dtype=torch.int32, device="cuda") if with_status else None
+            got = B.permute_noalloc(ids, E, capacity_factor=cf, x=x if with_x else None,
+                                    status_out=status)
+            ref = B.permute(ids, E, capacity_factor=cf, x=x if with_x else None)
+            torch.cuda.synchronize()
+            R = int(ref["offsets"][-1].item())
+            for name in ("counts", "offsets", "row_map"):
+                assert torch.equal(got[name], ref[name]), name
+            assert torch.equal(got["row_token"][:R], ref["row_token"][:R])
+            assert ("x_perm" in got) == with_x
+            if with_x:
+                assert torch.equal(got["x_perm"][:R], ref["x_perm"][:R])
+            if with_status:
+                assert int(status.item()) == B.OK
