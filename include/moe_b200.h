@@ -135,7 +135,15 @@ moe_status moe_permute_noalloc(const void* x, const int32_t* token_expert_idx,
  *   y_r = h_r W2[e]                     rounded to dt
  * T is the row count of x (for the gathered form).  y has R_max >= R rows;
  * rows >= R are not written.  R is read on the device from expert_offsets[E]
- * (no host synchronisation).  h lives in ws.                                */
+ * (no host synchronisation).  h lives in ws: at least
+ * moe_grouped_ffn_workspace_bytes(R_max, H, F, act, dt, 0) bytes.  With
+ * row_token, bf16 and a workspace of moe_grouped_ffn_workspace_bytes(..., 1)
+ * bytes, the rows are first copied into expert order inside ws and the dense
+ * kernel runs (faster than gathering four rows per TMA request inside the
+ * GEMM); a row_token entry outside [0, T) is then reported as
+ * MOE_ERR_INVALID_ARG through the device status and its row skipped.        */
+size_t moe_grouped_ffn_workspace_bytes(int R_max, int H, int F, moe_act act, moe_dtype dt,
+                                       int gathered);
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const void* x,
                            const void* w1, const void* w3, const void* w2,
                            const int32_t* expert_offsets, int R_max, int T, int H, int F,

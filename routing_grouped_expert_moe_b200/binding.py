@@ -35,6 +35,7 @@ _p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "moe_forward_host_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "moe_grouped_ffn_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_route": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p]),
     "moe_route_from_logits": (_i, [_p, _i, _i, _i, _p, _p, _p]),
     "moe_permute": (_i, [_p, _p, _i, _i, _i, _i, _f, _i, _p, _p, _p, _p, _p, _p, _sz, _p]),
@@ -264,7 +265,8 @@ def grouped_ffn(expert_offsets, w1, w3, w2, act="swiglu", x_perm=None, x=None, r
     if y is None:
         y = torch.empty(R_max, H, dtype=src.dtype, device=src.device)
     if ws is None:
-        ws = alloc_workspace(256 + R_max * F * src.element_size(), src.device)
+        ws = alloc_workspace(_lib.moe_grouped_ffn_workspace_bytes(
+            R_max, H, F, ACT[act], _dt(src), 1 if row_token is not None else 0), src.device)
     _check(_lib.moe_grouped_ffn(_ptr(x_perm), _ptr(row_token), _ptr(x), _ptr(w1), _ptr(w3),
                                 _ptr(w2), _ptr(expert_offsets), R_max, T, H, F, E, ACT[act],
                                 _dt(src), _ptr(y), _ptr(ws), ws.numel(), _stream()),

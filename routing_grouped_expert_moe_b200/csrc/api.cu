@@ -208,6 +208,17 @@ size_t moe_forward_host_workspace_bytes(int T, int H, int F, int E, int top_k, m
   return ws_layout(T, H, F, E, top_k, act, dt, true).total;
 }
 
+size_t moe_grouped_ffn_workspace_bytes(int R_max, int H, int F, moe_act act, moe_dtype dt,
+                                       int gathered) {
+  if (R_max < 0 || H <= 0 || F <= 0) return 0;
+  if (dt != MOE_F32 && dt != MOE_BF16) return 0;
+  const size_t eb = elem_bytes(dt);
+  size_t n = align_up(4) + (act == MOE_ACT_IDENTITY ? 0 : static_cast<size_t>(R_max) * F * eb);
+  if (gathered && dt == MOE_BF16 && act != MOE_ACT_IDENTITY)
+    n = align_up(n) + static_cast<size_t>(R_max) * H * eb;
+  return n;
+}
+
 moe_status moe_route(const void* x, const void* w_gate, const float* gate_bias, int T, int H,
                      int E, int top_k, moe_dtype dt, int32_t* topk_idx, float* topk_gate,
                      float* logits_out, moe_stream_t stream) {
@@ -300,7 +311,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
   if (gather && T <= 0) return MOE_ERR_INVALID_ARG;
   if (!index_range_ok(R_max, 1, H > F ? H : F)) return MOE_ERR_UNSUPPORTED;
   if (R_max == 0) return MOE_OK;
-  // h needs R_max * F elements after the status word.
+  // [status block | h: R_max x F | gathered rows: R_max x H (optional)]
   const size_t h_off = align_up(4);
   const size_t need = h_off + static_cast<size_t>(R_max) * F * elem_bytes(dt);
   if (act != MOE_ACT_IDENTITY && ws_bytes < need) return MOE_ERR_WORKSPACE;
@@ -309,6 +320,24 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
   int* status = at<int>(ws, 0);
   int* sched = at<int>(ws, kSchedInStatusBlock);
   if (launch_clear_status(status, s, sched, 2) != cudaSuccess) return MOE_ERR_CUDA;
+  // Gathered bf16 rows with room in ws: copy them into expert order once and
+  // run the dense kernel (a gathering TMA moves four rows per request).
+  const size_t xg_off = align_up(need);
+  const size_t xg_bytes = static_cast<size_t>(R_max) * H * elem_bytes(dt);
+  if (gather && dt == MOE_BF16 && act != MOE_ACT_IDENTITY && ws_bytes >= xg_off + xg_bytes) {
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.row_token = row_token;
+    g.E = E;
+    g.N = H;
+    g.R_max = R_max;
+    g.T = T;
+    g.out = at<void>(ws, xg_off);
+    g.status = status;
+    if (launch_copy_rows(x, g, elem_bytes(dt), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return run_ffn(at<void>(ws, xg_off), nullptr, x, w1, w3, w2, expert_offsets, R_max, T, H, F,
+                   E, act, dt, y, at<void>(ws, h_off), status, sched, s);
+  }
   return run_ffn(x_perm, row_token, x, w1, w3, w2, expert_offsets, R_max, T, H, F, E, act, dt, y,
                  at<void>(ws, h_off), status, sched, s);
 }

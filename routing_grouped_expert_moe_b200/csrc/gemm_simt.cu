@@ -136,15 +136,23 @@ cudaError_t launch_gemm_simt(int mode, const void* a_src, const void* b1, const 
   }
 }
 
-// Identity experts: out[r] = A[row_token[r]] (gather) or A[r], for r < offsets[E].
+// Rows of the expert segments: out[r] = A[row_token[r]] (gather) or A[r], for
+// offsets[0] <= r < offsets[E] (identity experts, and the gather ahead of the
+// dense GEMM).  A gathered row outside [0, T) is reported (invalid argument)
+// and skipped.
 __global__ void k_copy_rows(const uint8_t* __restrict__ A, const GemmArgs g, int row_bytes) {
   pdl_wait_and_trigger();
   const int R = min(g.offsets[g.E], g.R_max);
+  const int r0 = max(0, g.offsets[0]);
   const int vecs = row_bytes / 16;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int r = warp; r < R; r += nwarps) {
+  for (int r = r0 + warp; r < R; r += nwarps) {
     const int src_row = g.row_token ? g.row_token[r] : r;
+    if (g.row_token && (src_row < 0 || src_row >= g.T)) {
+      if (lane == 0) record_status(g.status, 1);
+      continue;
+    }
     const int4* src = reinterpret_cast<const int4*>(A + static_cast<size_t>(src_row) * row_bytes);
     int4* dst = reinterpret_cast<int4*>(static_cast<uint8_t*>(g.out) +
                                         static_cast<size_t>(r) * row_bytes);

@@ -73,20 +73,35 @@ __global__ void __launch_bounds__(kStatsThreads)
   }
 }
 
-// One thread per expert: counts from the router's per-tile histogram, the
-// probability sums from the per-tile partials, both in tile order.
-__global__ void k_route_stats_reduce(const int* __restrict__ tile_counts, int count_tiles,
-                                     const float* __restrict__ tile_prob, int prob_tiles, int T,
-                                     int E, int32_t* __restrict__ counts,
-                                     float* __restrict__ prob_mean) {
+// One CTA per expert: thread i sums tiles i, i + 256, ... in order, then a
+// fixed tree over the 256 partial sums (the same order on every run).
+__global__ void __launch_bounds__(kStatsThreads)
+    k_route_stats_reduce(const int* __restrict__ tile_counts, int count_tiles,
+                         const float* __restrict__ tile_prob, int prob_tiles, int T, int E,
+                         int32_t* __restrict__ counts, float* __restrict__ prob_mean) {
+  __shared__ int cs[kStatsThreads];
+  __shared__ float ps[kStatsThreads];
   pdl_wait_and_trigger();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int c = 0;
-    for (int j = 0; j < count_tiles; ++j) c += tile_counts[static_cast<size_t>(j) * E + e];
-    float p = 0.f;
-    for (int j = 0; j < prob_tiles; ++j) p += tile_prob[static_cast<size_t>(j) * E + e];
-    if (counts) counts[e] = c;
-    if (prob_mean) prob_mean[e] = p / static_cast<float>(T);
+  const int e = blockIdx.x;
+  int c = 0;
+  float p = 0.f;
+  for (int j = threadIdx.x; j < count_tiles; j += kStatsThreads)
+    c += tile_counts[static_cast<size_t>(j) * E + e];
+  for (int j = threadIdx.x; j < prob_tiles; j += kStatsThreads)
+    p += tile_prob[static_cast<size_t>(j) * E + e];
+  cs[threadIdx.x] = c;
+  ps[threadIdx.x] = p;
+  __syncthreads();
+  for (int w = kStatsThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      cs[threadIdx.x] += cs[threadIdx.x + w];
+      ps[threadIdx.x] += ps[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    if (counts) counts[e] = cs[0];
+    if (prob_mean) prob_mean[e] = ps[0] / static_cast<float>(T);
   }
 }
 
@@ -97,7 +112,8 @@ cudaError_t launch_route_stats(const float* logits, const int* tile_counts, int 
   cudaError_t err = launch_kernel(k_route_prob_tiles, dim3(prob_tiles), dim3(kStatsThreads), 0, s,
                                   1, logits, T, E, tile_prob);
   if (err != cudaSuccess) return err;
-  return launch_kernel(k_route_stats_reduce, dim3(1), dim3(256), 0, s, 1, tile_counts, count_tiles,
+  return launch_kernel(k_route_stats_reduce, dim3(E), dim3(kStatsThreads), 0, s, 1, tile_counts,
+                       count_tiles,
                        static_cast<const float*>(tile_prob), prob_tiles, T, E, counts, prob_mean);
 }
 

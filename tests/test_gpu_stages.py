@@ -193,6 +193,7 @@ def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
     rt[:R] = torch.from_numpy(perm["row_token"].astype(np.int32))
     esz = 2 if dtype == "bf16" else 4
     y = Guarded((R_max, H), dt)
+    # the smallest workspace: gathered rows are read by the GEMM itself
     ws = guarded_workspace(256 + R_max * F * esz)
     if gather:
         B().grouped_ffn(offs, w1.cuda(), None if w3 is None else w3.cuda(), w2.cuda(), act,
@@ -208,6 +209,29 @@ def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
     assert rel_err(got, ref) <= TOL[dtype]
     y.check("y")
     y.untouched(R * H * esz, R_max * H * esz, "y rows past R")
+    ws.check("workspace")
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_grouped_ffn_gather_with_room_equals_dense(act):
+    """With room for the gathered rows in ws, the gathered form copies them into
+    expert order and runs the dense kernel: bit-identical to passing x_perm."""
+    E, rows, H, F = 5, [512, 640, 383, 0, 129], 384, 512
+    dt, x, w1, w3, w2, perm = _ffn_case("bf16", act, E, rows, H, F)
+    offs = torch.from_numpy(perm["offsets"].astype(np.int32)).cuda()
+    rt = torch.from_numpy(perm["row_token"].astype(np.int32)).cuda()
+    R = perm["R"]
+    w3c = None if w3 is None else w3.cuda()
+    ws = guarded_workspace(B()._lib.moe_grouped_ffn_workspace_bytes(R, H, F, B().ACT[act],
+                                                                    B().BF16, 1))
+    yg = Guarded((R, H), dt)
+    B().grouped_ffn(offs, w1.cuda(), w3c, w2.cuda(), act, x=x.cuda(), row_token=rt, ws=ws.t,
+                    y=yg.t)
+    x_perm = x[torch.from_numpy(perm["row_token"])].contiguous().cuda()
+    yd = B().grouped_ffn(offs, w1.cuda(), w3c, w2.cuda(), act, x_perm=x_perm)
+    assert B().device_status(ws.t) == B().OK
+    assert torch.equal(yg.t, yd)
+    yg.check("y")
     ws.check("workspace")
 
 
