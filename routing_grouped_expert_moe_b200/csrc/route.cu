@@ -102,7 +102,9 @@ __device__ void route_select_and_count(const float* logits_s, int ls_stride, int
 
 // ----------------------------------------------------------------------------
 // SIMT router (fp32 storage, or bf16 with an expert count that is not a
-// multiple of 8).  One warp per token, lanes over experts, H in order.
+// multiple of 8).  One warp per token; lane l takes h = l, l + 32, ... (x read
+// coalesced), experts in chunks of 8 accumulated per lane, then a warp
+// butterfly per chunk (fixed order: deterministic).
 // ----------------------------------------------------------------------------
 constexpr int kSimtBT = 32;
 
@@ -130,21 +132,25 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_simt(RouteArgs a) {
   for (int lt = warp; lt < kSimtBT; lt += kRouteThreads / 32) {
     const int t = token0 + lt;
     if (t >= a.T) continue;
-    float acc[8];
+    const Tin* xr = x + static_cast<size_t>(t) * a.H;
+    for (int e0 = 0; e0 < a.E; e0 += 8) {
+      float acc[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    for (int h = 0; h < a.H; ++h) {
-      const float xv = to_f<Tin>(x[static_cast<size_t>(t) * a.H + h]);
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      for (int h = lane; h < a.H; h += 32) {
+        const float xv = to_f<Tin>(xr[h]);
+        const Tin* wr = wg + static_cast<size_t>(h) * a.E + e0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (e0 + j < a.E) acc[j] = fmaf(xv, to_f<Tin>(wr[j]), acc[j]);
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        if (e < a.E) acc[j] = fmaf(xv, to_f<Tin>(wg[static_cast<size_t>(h) * a.E + e]), acc[j]);
-      }
-    }
+        float v = acc[j];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      if (e < a.E) lg[lt * E_STR + e] = acc[j];
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == j && e0 + j < a.E) lg[lt * E_STR + e0 + j] = v;
+      }
     }
   }
   __syncthreads();
