@@ -135,13 +135,16 @@ moe_status moe_permute_noalloc(const void* x, const int32_t* token_expert_idx,
  *   y_r = h_r W2[e]                     rounded to dt
  * T is the row count of x (for the gathered form).  y has R_max >= R rows;
  * rows >= R are not written.  R is read on the device from expert_offsets[E]
- * (no host synchronisation).  h lives in ws: at least
- * moe_grouped_ffn_workspace_bytes(R_max, H, F, act, dt, 0) bytes.  With
- * row_token, bf16 and a workspace of moe_grouped_ffn_workspace_bytes(..., 1)
- * bytes, the rows are first copied into expert order inside ws and the dense
- * kernel runs (faster than gathering four rows per TMA request inside the
- * GEMM); a row_token entry outside [0, T) is then reported as
- * MOE_ERR_INVALID_ARG through the device status and its row skipped.        */
+ * (no host synchronisation).  h lives in ws, after a 256-byte status block:
+ * the call needs 256 + R_max * F * sizeof(dt) bytes (MOE_ERR_WORKSPACE
+ * below that; 256 for MOE_ACT_IDENTITY).  moe_grouped_ffn_workspace_bytes
+ * returns a size with room for two optional parts, used when ws_bytes covers
+ * them: (1) with row_token, bf16 and gathered != 0, the rows copied into
+ * expert order, after which the dense kernel runs (faster than gathering
+ * four rows per TMA request inside the GEMM); a row_token entry outside
+ * [0, T) is then reported as MOE_ERR_INVALID_ARG through the device status
+ * and its row skipped; (2) for bf16, fp32 partial sums (40 MiB) and tickets
+ * that let the GEMMs cut their last partial wave of tiles along K.         */
 size_t moe_grouped_ffn_workspace_bytes(int R_max, int H, int F, moe_act act, moe_dtype dt,
                                        int gathered);
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const void* x,
@@ -348,7 +351,8 @@ moe_status moe_workspace_section(int T, int H, int F, int E, int top_k, moe_act 
  * when the library loads); 1 = row tiles of 128 rows, one CTA each; 2 = row
  * tiles of 256 rows on CTA pairs; 3 = token-as-N tiles on CTA pairs (the
  * tokens of an expert as the MMA's N; dense A rows only, gathered rows use
- * the automatic choice).  Returns MOE_ERR_INVALID_ARG for other values.
+ * the automatic choice); 4 = the same without cutting the last partial
+ * wave of tiles along K.  Returns MOE_ERR_INVALID_ARG for other values.
  * Not synchronised with calls running on other host threads.               */
 moe_status moe_set_gemm_variant(int variant);
 

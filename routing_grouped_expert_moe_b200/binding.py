@@ -517,7 +517,8 @@ def device_status(ws) -> int:
 
 WS_SECTIONS = {"topk_idx": 0, "topk_gate": 1, "counts": 2, "offsets": 3, "row_token": 4,
                "row_map": 5, "x_perm": 6, "h": 7, "y": 8}
-GEMM_VARIANTS = {"auto": 0, "rows128": 1, "rows256_pair": 2, "tokens_pair": 3}
+GEMM_VARIANTS = {"auto": 0, "rows128": 1, "rows256_pair": 2, "tokens_pair": 3,
+                 "tokens_pair_nosplit": 4}
 
 
 def workspace_section(ws, name, T, H, F, E, top_k, act="swiglu", dtype=torch.bfloat16):

@@ -32,6 +32,7 @@ Tuning read_tuning() {
   t.route_shallow = env_int("MOE_ROUTE_DEEP", 1) == 0;
   t.tokn_nacc = env_int("MOE_TOKN_NACC", 0);
   t.tokn_bk = env_int("MOE_TOKN_BK", 0);
+  t.tokn_split = env_int("MOE_TOKN_SPLIT", 2);
   return t;
 }
 // Initialised when the library is loaded.
@@ -65,14 +66,20 @@ int num_sms_current() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace: [status | topk_idx | topk_gate | tile_counts | sched + tickets | partials |
-//             counts | offsets | row_token | row_map | x_perm | h | y | x_stage | out_stage]
+// Workspace: [status | topk_idx | topk_gate | tile_counts | sched + tickets + split tickets |
+//             partials | counts | offsets | row_token | row_map | x_perm | h | y | split sums |
+//             x_stage | out_stage]
 // sched: the grouped GEMMs' tile counters (kSchedCounters ints), directly
-// followed by the router's tickets, so one clear covers both.
+// followed by the router's tickets and the two GEMMs' K-split tickets, so one
+// clear covers all three.
 constexpr int kSchedCounters = 4;
+constexpr int kSplitTicketInts = kSplitTiles * kSplitTileTickets;  // per GEMM
+constexpr size_t kSplitSumBytes = static_cast<size_t>(kSplitUnits) * kSplitUnitFloats * 4;
 struct WsLayout {
-  size_t status, topk_idx, topk_gate, tile_counts, sched, tickets, partials, counts, offsets,
-      row_token, row_map, x_perm, h, y, x_stage, out_stage, logits, n_sel, total;
+  size_t status, topk_idx, topk_gate, tile_counts, sched, tickets, split_tickets, partials,
+      counts, offsets, row_token, row_map, x_perm, h, y, split_sums, x_stage, out_stage, logits,
+      n_sel, total;
+  int clear_ints;  // ints zeroed from sched on
 };
 
 // Workspaces that begin with the status word's 256-byte block keep the GEMMs'
@@ -92,7 +99,9 @@ WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt,
   L.tile_counts = o; o = align_up(o + tiles * E * 4);
   L.sched = o;
   L.tickets = o + kSchedCounters * 4;
-  o = align_up(L.tickets + (static_cast<size_t>(T) / 128 + 1) * 4);
+  L.split_tickets = L.tickets + (static_cast<size_t>(T) / 128 + 1) * 4;
+  L.clear_ints = kSchedCounters + T / 128 + 1 + 2 * kSplitTicketInts;
+  o = align_up(L.split_tickets + 2 * kSplitTicketInts * 4);
   L.partials = o;    o = align_up(o + static_cast<size_t>(kRouteMaxCtas) * 128 * E * 4);
   L.counts = o;      o = align_up(o + static_cast<size_t>(E) * 4);
   L.offsets = o;     o = align_up(o + static_cast<size_t>(E + 1) * 4);
@@ -101,6 +110,8 @@ WsLayout ws_layout(int T, int H, int F, int E, int k, moe_act act, moe_dtype dt,
   L.x_perm = o;      o = align_up(o + R * H * eb);
   L.h = o;           o = align_up(o + (act == MOE_ACT_IDENTITY ? 0 : R * F * eb));
   L.y = o;           o = align_up(o + R * H * eb);
+  const bool tc = dt == MOE_BF16 && act != MOE_ACT_IDENTITY;  // tensor-core experts
+  L.split_sums = o;  o = align_up(o + (tc ? kSplitSumBytes : 0));
   if (host_stage) {
     L.x_stage = o;   o = align_up(o + static_cast<size_t>(T) * H * eb);
     L.out_stage = o; o = align_up(o + static_cast<size_t>(T) * H * eb);
@@ -143,11 +154,14 @@ int capacity_of(float cf, int T, int k, int E) {
 cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // Grouped FFN on prepared buffers (shared by moe_grouped_ffn and moe_forward).
-// sched: two zeroed tile counters (GEMM-1, GEMM-2).
+// sched: two zeroed tile counters (GEMM-1, GEMM-2).  split_sums (kSplitSumBytes)
+// and split_tickets (2 x kSplitTicketInts zeroed ints), or nulls: room for the
+// GEMMs' K-split tail.
 moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, const void* w1,
                    const void* w3, const void* w2, const int32_t* offsets, int R_max, int T,
                    int H, int F, int E, moe_act act, moe_dtype dt, void* y, void* h, int* status,
-                   int* sched, cudaStream_t s, cudaEvent_t mid_event = nullptr) {
+                   int* sched, float* split_sums, int* split_tickets, cudaStream_t s,
+                   cudaEvent_t mid_event = nullptr) {
   const int nsm = num_sms_current();
   const bool gather = row_token != nullptr;
   const void* a_src = gather ? x : x_perm;
@@ -158,6 +172,11 @@ moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, 
   g.R_max = R_max;
   g.T = T;
   g.status = status;
+  if (split_sums != nullptr && split_tickets != nullptr) {
+    g.split_ws = split_sums;
+    g.split_units = kSplitUnits;
+    g.split_tiles = kSplitTiles;
+  }
   if (act == MOE_ACT_IDENTITY) {
     g.row_token = row_token;
     g.N = H;
@@ -173,6 +192,7 @@ moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, 
   g.K = H;
   g.out = h;
   g.sched = sched;
+  g.split_tickets = g.split_ws ? split_tickets : nullptr;
   cudaError_t err;
   if (dt == MOE_BF16)
     err = launch_gemm_tc(mode1, gather, a_src, a_rows, w1, w3, g, nsm, s);
@@ -186,6 +206,7 @@ moe_status run_ffn(const void* x_perm, const int32_t* row_token, const void* x, 
   g.K = F;
   g.out = y;
   g.sched = sched + 1;
+  g.split_tickets = g.split_ws ? split_tickets + kSplitTicketInts : nullptr;
   if (dt == MOE_BF16)
     err = launch_gemm_tc(2, false, h, R_max, w2, nullptr, g, nsm, s);
   else
@@ -213,9 +234,10 @@ size_t moe_grouped_ffn_workspace_bytes(int R_max, int H, int F, moe_act act, moe
   if (R_max < 0 || H <= 0 || F <= 0) return 0;
   if (dt != MOE_F32 && dt != MOE_BF16) return 0;
   const size_t eb = elem_bytes(dt);
+  const bool tc = dt == MOE_BF16 && act != MOE_ACT_IDENTITY;
   size_t n = align_up(4) + (act == MOE_ACT_IDENTITY ? 0 : static_cast<size_t>(R_max) * F * eb);
-  if (gathered && dt == MOE_BF16 && act != MOE_ACT_IDENTITY)
-    n = align_up(n) + static_cast<size_t>(R_max) * H * eb;
+  if (gathered && tc) n = align_up(n) + static_cast<size_t>(R_max) * H * eb;
+  if (tc) n = align_up(n) + align_up(2 * kSplitTicketInts * 4) + kSplitSumBytes;
   return n;
 }
 
@@ -311,7 +333,8 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
   if (gather && T <= 0) return MOE_ERR_INVALID_ARG;
   if (!index_range_ok(R_max, 1, H > F ? H : F)) return MOE_ERR_UNSUPPORTED;
   if (R_max == 0) return MOE_OK;
-  // [status block | h: R_max x F | gathered rows: R_max x H (optional)]
+  // [status block | h: R_max x F | gathered rows: R_max x H (optional) |
+  //  K-split tickets + sums (optional)]; the optional parts are used when ws has room
   const size_t h_off = align_up(4);
   const size_t need = h_off + static_cast<size_t>(R_max) * F * elem_bytes(dt);
   if (act != MOE_ACT_IDENTITY && ws_bytes < need) return MOE_ERR_WORKSPACE;
@@ -319,12 +342,21 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
   cudaStream_t s = as_stream(stream);
   int* status = at<int>(ws, 0);
   int* sched = at<int>(ws, kSchedInStatusBlock);
-  if (launch_clear_status(status, s, sched, 2) != cudaSuccess) return MOE_ERR_CUDA;
-  // Gathered bf16 rows with room in ws: copy them into expert order once and
-  // run the dense kernel (a gathering TMA moves four rows per request).
+  const bool tc = dt == MOE_BF16 && act != MOE_ACT_IDENTITY;
   const size_t xg_off = align_up(need);
   const size_t xg_bytes = static_cast<size_t>(R_max) * H * elem_bytes(dt);
-  if (gather && dt == MOE_BF16 && act != MOE_ACT_IDENTITY && ws_bytes >= xg_off + xg_bytes) {
+  const bool gather_dense = gather && tc && ws_bytes >= xg_off + xg_bytes;
+  const size_t sp_off = gather_dense ? align_up(xg_off + xg_bytes) : xg_off;
+  const size_t sp_tickets_bytes = align_up(2 * kSplitTicketInts * 4);
+  const bool split = tc && ws_bytes >= sp_off + sp_tickets_bytes + kSplitSumBytes;
+  int* sp_tickets = split ? at<int>(ws, sp_off) : nullptr;
+  float* sp_sums = split ? at<float>(ws, sp_off + sp_tickets_bytes) : nullptr;
+  if (launch_clear_status(status, s, sched, 2, sp_tickets, split ? 2 * kSplitTicketInts : 0) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  // Gathered bf16 rows with room in ws: copy them into expert order once and
+  // run the dense kernel (a gathering TMA moves four rows per request).
+  if (gather_dense) {
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.row_token = row_token;
@@ -336,10 +368,10 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
     g.status = status;
     if (launch_copy_rows(x, g, elem_bytes(dt), s) != cudaSuccess) return MOE_ERR_CUDA;
     return run_ffn(at<void>(ws, xg_off), nullptr, x, w1, w3, w2, expert_offsets, R_max, T, H, F,
-                   E, act, dt, y, at<void>(ws, h_off), status, sched, s);
+                   E, act, dt, y, at<void>(ws, h_off), status, sched, sp_sums, sp_tickets, s);
   }
   return run_ffn(x_perm, row_token, x, w1, w3, w2, expert_offsets, R_max, T, H, F, E, act, dt, y,
-                 at<void>(ws, h_off), status, sched, s);
+                 at<void>(ws, h_off), status, sched, sp_sums, sp_tickets, s);
 }
 
 moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
@@ -560,8 +592,7 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   auto mark = [&](int i) { return ev && ev[i] ? cudaEventRecord(ev[i], s) : cudaSuccess; };
   int* sched = at<int>(ws, L.sched);
   int* tickets = at<int>(ws, L.tickets);
-  if (launch_clear_status(status, s, sched, kSchedCounters + T / 128 + 1) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (launch_clear_status(status, s, sched, L.clear_ints) != cudaSuccess) return MOE_ERR_CUDA;
   // 1. route (+ per-tile histogram)
   if (mark(0) != cudaSuccess) return MOE_ERR_CUDA;
   RouteArgs ra{};
@@ -611,8 +642,11 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   // 3. experts
   const int R_max = T * top_k;
   void* y = at<void>(ws, L.y);
+  const bool tc = bf16 && act != MOE_ACT_IDENTITY;
   st = run_ffn(x_perm, bf16 ? nullptr : row_token, x, w1, w3, w2, offsets, R_max, T, H, F, E, act,
-               dt, y, at<void>(ws, L.h), status, sched, s, ev ? ev[4] : nullptr);
+               dt, y, at<void>(ws, L.h), status, sched,
+               tc ? at<float>(ws, L.split_sums) : nullptr,
+               tc ? at<int>(ws, L.split_tickets) : nullptr, s, ev ? ev[4] : nullptr);
   if (st != MOE_OK) return st;
   if (mark(5) != cudaSuccess) return MOE_ERR_CUDA;
   // 4. combine
@@ -824,7 +858,7 @@ moe_status moe_workspace_section(int T, int H, int F, int E, int top_k, moe_act 
 }
 
 moe_status moe_set_gemm_variant(int variant) {
-  if (variant < 0 || variant > 3) return MOE_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 4) return MOE_ERR_INVALID_ARG;
   moe::g_gemm_variant.store(variant, std::memory_order_relaxed);
   return MOE_OK;
 }

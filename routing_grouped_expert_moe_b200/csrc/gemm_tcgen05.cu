@@ -284,7 +284,7 @@ static cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b1, const 
 // tile, as measured) is lower.  The tuning variant forces one.
 static int choose_variant(int mode, bool gather, const GemmArgs& g, int num_sms) {
   const int forced = gemm_variant();
-  if (forced == 3 && !gather) return 3;
+  if (forced >= 3 && !gather) return 3;  // 4: token-as-N without the K-split tail
   if (forced == 1 || forced == 2) return forced;
   if (!gather) return 3;
   const double a = static_cast<double>(g.R_max) / g.E;

@@ -20,6 +20,18 @@
 // accumulator so the epilogue of a tile overlaps the next tile's main loop;
 // NACC = 2 (SwiGLU: W1 and W3) fills the 512 TMEM columns with one tile.
 //
+// K-split tail: a tile's time is set by its number of pipeline stages (the
+// loads' latency under load, not their bytes, paces a stage), so tiles of
+// one launch take about the same time and the last wave, total mod the CTA
+// pairs, runs on a fraction of the GPU.  When at most half the pairs are
+// left for it (and the host asks for it: the SwiGLU GEMM-1), those last
+// tiles are cut along K into two parts.  Each part
+// writes its fp32 accumulators to the workspace, then counts itself in on a
+// ticket per epilogue warp; the part that comes second adds the other's sums
+// to its own (fp32 addition of two terms is commutative, so the result does
+// not depend on which part finished first) and runs the activation and the
+// stores.  No part waits for another.
+//
 // Tiles are taken from a global counter (dynamic schedule: token groups of
 // different sizes take different times).  The first CTA's producer takes the
 // next tile and passes its index to the other CTA's producer through a mailbox
@@ -81,6 +93,14 @@ __host__ __device__ constexpr TokRows tok_rows(int half_n) {
 
 struct TokTile {
   int e, row0, rows, n, col0;
+  int kb0, kb1;     // k-blocks of this part
+  int unit;         // K-split part index over the split tiles (-1: a whole tile)
+  int part, stile;  // part within its tile, split tile index
+};
+
+// Launch-wide schedule: tiles [0, t0) whole, tiles [t0, total) in S parts each.
+struct TokSplit {
+  int t0, S, units;
 };
 
 // Tile tau -> (expert, token group, output-column block); groups vary fastest,
@@ -88,7 +108,15 @@ struct TokTile {
 // read of the weights hits L2.
 __device__ __forceinline__ TokTile decode_tok(int tau, const int* prefix, const int* seg_start,
                                              const int* seg_rows, const int* grp_rows,
-                                             const int* ngrp, int E, int cols_per_tile) {
+                                             const int* ngrp, int E, int cols_per_tile,
+                                             const TokSplit& sp, int num_kb) {
+  int unit = -1, part = 0, stile = -1;
+  if (tau >= sp.t0) {  // a K-split part
+    unit = tau - sp.t0;
+    stile = unit / sp.S;
+    part = unit - stile * sp.S;
+    tau = sp.t0 + stile;
+  }
   int lo = 0, hi = E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -105,6 +133,11 @@ __device__ __forceinline__ TokTile decode_tok(int tau, const int* prefix, const 
   t.rows = min(q, seg_rows[lo] - g * q);
   t.n = (t.rows + 15) & ~15;
   t.col0 = mb * cols_per_tile;
+  t.unit = unit;
+  t.part = part;
+  t.stile = stile;
+  t.kb0 = unit < 0 ? 0 : (part * num_kb) / sp.S;
+  t.kb1 = unit < 0 ? num_kb : ((part + 1) * num_kb) / sp.S;
   return t;
 }
 
@@ -193,6 +226,7 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
   __shared__ int s_seg_rows[kMaxE];
   __shared__ int s_grp_rows[kMaxE];
   __shared__ int s_ngrp[kMaxE];
+  __shared__ TokSplit s_split;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -255,6 +289,19 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
     }
     if (lane == 0) {
       s_prefix[0] = 0;
+      // the last partial wave (total mod pairs tiles) in two parts along K, each
+      // part at least 2 k-blocks, within the workspace's capacity
+      const int total = carry;
+      const int pairs = static_cast<int>(gridDim.x) >> 1;
+      const int rem = pairs > 0 ? total % pairs : 0;
+      int S = 1;
+      if (args.split_max >= 2 && args.split_ws != nullptr && args.split_tickets != nullptr &&
+          rem > 0 && 2 * rem <= pairs && rem <= args.split_tiles && 2 * rem <= args.split_units &&
+          num_kb >= 4)
+        S = 2;
+      s_split.S = S > 1 ? S : 1;
+      s_split.t0 = S > 1 ? total - rem : total;
+      s_split.units = S > 1 ? total - rem + rem * S : total;
       tma_prefetch_desc(&tmX32);
       tma_prefetch_desc(&tmX64);
       tma_prefetch_desc(&tmX128);
@@ -270,7 +317,8 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
-  const int total = s_prefix[E];
+  const TokSplit sp = s_split;
+  const int total = sp.units;  // whole tiles and K-split parts
   volatile int* abort_flag = &abort_s;
   volatile int* vs_tile = s_tile;
   volatile int* vmb_tile = mb_tile;
@@ -326,7 +374,7 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
         }
         if (tau < 0) break;
         const TokTile ti = decode_tok(tau, s_prefix, s_seg_start, s_seg_rows, s_grp_rows, s_ngrp, E,
-                                      C::COLS_PER_TILE);
+                                      C::COLS_PER_TILE, sp, num_kb);
         const int half_n = ti.n >> 1;
         // this CTA's token rows: one box of 32, 64 or 128 rows, or 64 + 32
         const TokRows xr = tok_rows(half_n);
@@ -337,7 +385,7 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
         const uint32_t tx = 2u * static_cast<uint32_t>(C::A_BYTES + (BK / 64) * rows_ld * 128);
         const int wcol = ti.col0 + 128 * static_cast<int>(rank);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++g) {
           if (g % C::PROD != static_cast<uint32_t>(p)) continue;
           const int stage = static_cast<int>(g % C::STAGES);
           const uint32_t phase = (g / C::STAGES) & 1u;
@@ -384,14 +432,14 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
         if (!ok || tau < 0) break;
         if (lane == 0) {
           const TokTile ti = decode_tok(tau, s_prefix, s_seg_start, s_seg_rows, s_grp_rows,
-                                        s_ngrp, E, C::COLS_PER_TILE);
+                                        s_ngrp, E, C::COLS_PER_TILE, sp, num_kb);
           const uint32_t idesc = idesc_bf16_f32(256, ti.n, true, false);
           if (!mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, args.status)) {
             ok = false;
           } else {
             tc_fence_after();
             const uint32_t d0 = tmem_base + static_cast<uint32_t>(NACC == 2 ? 0 : acc * 256);
-            for (int kb = 0; kb < num_kb; ++kb) {
+            for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
               if (!mbar_wait(&full_bar[stage], phase, abort_flag, args.status)) { ok = false; break; }
               tc_fence_after();
               const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -407,7 +455,8 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
                   // weights: MN-major, 64-column boxes W_BOX apart, K step of 16 rows = 2 KB
                   const uint64_t wdesc =
                       smem_desc(a_base + j * C::W_BYTES + kk * 2048, C::W_BOX, 1024);
-                  umma_f16_pair(d0 + j * 256, wdesc, xdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                  umma_f16_pair(d0 + j * 256, wdesc, xdesc, idesc,
+                                (kb != ti.kb0 || kk != 0) ? 1u : 0u);
                 }
               }
               umma_commit_pair_both(&empty_bar[stage]);
@@ -438,7 +487,7 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
       const int tau = next_tile(i, ok);
       if (!ok || tau < 0) break;
       const TokTile ti = decode_tok(tau, s_prefix, s_seg_start, s_seg_rows, s_grp_rows, s_ngrp, E,
-                                    C::COLS_PER_TILE);
+                                    C::COLS_PER_TILE, sp, num_kb);
       int w = 1;
       if (lane == 0)
         w = mbar_wait_polite<true>(&tfull_bar[acc], acc_phase, abort_flag, args.status,
@@ -449,10 +498,76 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
                               static_cast<uint32_t>(NACC == 2 ? 0 : acc * 256);
       const int nch = (ti.n + 31) >> 5;
       const int colw = ti.col0 + 128 * static_cast<int>(rank) + q * 32;  // this warp's 32 columns
+      constexpr int NOUT = MODE == 1 ? 1 : NACC;          // outputs per chunk
+      constexpr int NP = (MODE == 1 || NACC == 2) ? 2 : 1;  // accumulators per chunk
+      // A K-split part (two per tile): its fp32 sums for this warp's chunks,
+      // [chunk / 2][acc][token / 4][lane][token % 4], so that a warp moves 512
+      // contiguous bytes per float4 access.
+      const size_t wslot = static_cast<size_t>((static_cast<int>(rank) * 8 + (warp - 2)) * 4 * 2 * 1024);
+      bool emit = true;
+      if (ti.unit >= 0) {
+        float* mine = args.split_ws + static_cast<size_t>(ti.unit) * kSplitUnitFloats + wslot;
 #pragma unroll 1
-      for (int c = half; c < nch; c += 2) {
+        for (int c = half; c < nch; c += 2) {
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            float v[32];
+            tmem_ld32(t_lane + j * 256 + c * 32, v);
+            tmem_ld_wait();
+            reg_fence32(v);
+            float4* dst = reinterpret_cast<float4*>(mine + ((c >> 1) * 2 + j) * 1024) + lane;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              __stcg(dst + i * 32, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+          }
+        }
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0)
+          last = atomicAdd(&args.split_tickets[ti.stile * kSplitTileTickets +
+                                               static_cast<int>(rank) * 8 + (warp - 2)],
+                           1) == 1;
+        emit = __shfl_sync(0xffffffffu, last, 0) != 0;
+        if (emit) __threadfence();  // the other part's sums are visible past the ticket
+      }
+      if (ti.unit >= 0 && emit) {
+        // The second part folds the first one's sums into its accumulators
+        // (own + other: fp32 addition of two terms is commutative, so the
+        // result does not depend on which part finished first).
+        const float* other = args.split_ws + static_cast<size_t>(ti.unit ^ 1) * kSplitUnitFloats + wslot;
+        const int nu = ((nch - half + 1) >> 1) * NP;  // this warp's (chunk, accumulator) pairs
+        auto load_other = [&](float4 (&o)[8], int k) {
+          const int c = half + 2 * (k / NP);
+          const float4* src =
+              reinterpret_cast<const float4*>(other + ((c >> 1) * 2 + k % NP) * 1024) + lane;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = __ldcg(src + i * 32);
+        };
+#pragma unroll 1
+        for (int k = 0; k < nu; ++k) {
+          float4 cur[8];
+          load_other(cur, k);
+          const int c = half + 2 * (k / NP);
+          const uint32_t ta = t_lane + (k % NP) * 256 + c * 32;
+          float v[32];
+          tmem_ld32(ta, v);
+          tmem_ld_wait();
+          reg_fence32(v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] += cur[i].x;
+            v[4 * i + 1] += cur[i].y;
+            v[4 * i + 2] += cur[i].z;
+            v[4 * i + 3] += cur[i].w;
+          }
+          tmem_st32(ta, v);
+        }
+        tmem_st_wait();
+      }
+#pragma unroll 1
+      for (int c = half; emit && c < nch; c += 2) {
         const int vt = min(32, ti.rows - c * 32);  // tokens of this chunk inside the group
-        constexpr int NOUT = MODE == 1 ? 1 : NACC;
 #pragma unroll
         for (int j = 0; j < NOUT; ++j) {
           float v[32], u[32];
@@ -508,8 +623,14 @@ static cudaError_t launch_tokn_bk(int bk, const CUtensorMap* x, const CUtensorMa
 }
 
 cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void* b1,
-                             const void* b3, const GemmArgs& g, int num_sms, cudaStream_t s) {
-  if (g.sched == nullptr) return cudaErrorInvalidValue;
+                             const void* b3, const GemmArgs& g_in, int num_sms, cudaStream_t s) {
+  if (g_in.sched == nullptr) return cudaErrorInvalidValue;
+  GemmArgs g = g_in;
+  // K-split tail: measured on the Mixtral-shaped, 128-expert and 32-expert
+  // layers, the SwiGLU GEMM-1 (one accumulator pair, epilogue not overlapped)
+  // gains 1-2.5%; the GELU and down-projection GEMMs (double-buffered) lose
+  // up to 1%, so they keep whole tiles.
+  g.split_max = (mode == 1 && gemm_variant() != 4) ? tuning().tokn_split : 1;
   // Tile shape per GEMM (measured on the Mixtral-shaped and page-1 layers):
   // SwiGLU keeps two accumulators (W1, W3) and 4 stages of K = 64; GELU one
   // double-buffered accumulator and 3 stages of K = 128; the down-projection

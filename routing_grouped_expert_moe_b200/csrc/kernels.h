@@ -22,6 +22,7 @@ struct Tuning {
   bool route_shallow = false;   // MOE_ROUTE_DEEP=0: keep the router's shallow ring
   int tokn_nacc = 0;            // MOE_TOKN_NACC=1|2: force the accumulators per tile (GELU, down)
   int tokn_bk = 0;              // MOE_TOKN_BK=64|128: force the K per pipeline stage
+  int tokn_split = 2;           // MOE_TOKN_SPLIT=1: no K-split of the last partial wave
 };
 const Tuning& tuning();
 // Grouped-GEMM kernel choice: 0 automatic, 1 | 2 | 3 forced (moe_set_gemm_variant;
@@ -128,7 +129,19 @@ struct GemmArgs {
   int* status;
   int* sched;                // tile counter of the dynamic schedule (zero before the launch)
   int epi_sleep_ns;          // epilogue warps' sleep between polls of the accumulator barrier
+  // K-split of the last partial wave of tiles (token-as-N kernel; null: off)
+  float* split_ws;           // split_units x kSplitUnitFloats fp32 partial sums
+  int* split_tickets;        // split_tiles x kSplitTileTickets tickets, zero before the launch
+  int split_units, split_tiles;
+  int split_max;             // 2: cut the last partial wave of tiles in two along K; 1: no
 };
+
+// One K-split part's partial sums: 2 CTAs x 8 epilogue warps x 4 chunks of 32
+// tokens x 2 accumulators x 32 tokens x 32 columns.
+constexpr int kSplitUnitFloats = 2 * 8 * 4 * 2 * 32 * 32;
+constexpr int kSplitTileTickets = 16;  // one per epilogue warp of the pair
+constexpr int kSplitTiles = 128;       // split tiles per GEMM (at most the CTA pairs - 1)
+constexpr int kSplitUnits = 80;        // split parts per GEMM (at most the CTA pairs)
 
 // bf16 tensor-core (tcgen05) path. a_src: x_perm/h rows (dense) or x (gather).
 cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows, const void* b1,
@@ -177,6 +190,7 @@ cudaError_t launch_selftest_bounded_wait(int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- misc
 // Clears the status word and n counters (the router's tickets).
-cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters = nullptr, int n = 0);
+cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters = nullptr, int n = 0,
+                                int* counters2 = nullptr, int n2 = 0);
 
 }  // namespace moe

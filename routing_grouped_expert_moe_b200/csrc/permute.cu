@@ -202,16 +202,19 @@ cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s) {
                        0, s, 1, a);
 }
 
-__global__ void k_clear_status(int* status, int* counters, int n) {
+__global__ void k_clear_status(int* status, int* counters, int n, int* counters2, int n2) {
   pdl_wait_and_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
     counters[i] = 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += gridDim.x * blockDim.x)
+    counters2[i] = 0;
 }
 
-cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters, int n) {
-  return launch_kernel(k_clear_status, dim3(1), dim3(256), 0, s, 1, status, counters,
-                       counters ? n : 0);
+cudaError_t launch_clear_status(int* status, cudaStream_t s, int* counters, int n, int* counters2,
+                                int n2) {
+  return launch_kernel(k_clear_status, dim3(1), dim3(512), 0, s, 1, status, counters,
+                       counters ? n : 0, counters2, counters2 ? n2 : 0);
 }
 
 }  // namespace moe

@@ -101,7 +101,8 @@ SMALL = [
 
 
 @pytest.mark.parametrize("oracle", ["numpy", "cpp"])
-@pytest.mark.parametrize("variant", ["rows128", "rows256_pair", "tokens_pair"])
+@pytest.mark.parametrize("variant", ["rows128", "rows256_pair", "tokens_pair",
+                                     "tokens_pair_nosplit"])
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_forward_small_full_compare(cfg, variant, oracle, gemm_variant):
     if cfg.dtype == "f32" and variant != "rows128":

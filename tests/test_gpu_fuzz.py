@@ -42,7 +42,8 @@ def test_forward_fuzz(cfg, gemm_variant):
     """Each case on one of the three bf16 GEMM kernels in turn; outputs and the
     workspace sentinel-guarded, rows past R untouched."""
     from routing_grouped_expert_moe_b200 import binding as B
-    gemm_variant(["tokens_pair", "rows128", "rows256_pair"][int(cfg.name[4:]) % 3])
+    gemm_variant(["tokens_pair", "rows128", "rows256_pair", "tokens_pair_nosplit"]
+                 [int(cfg.name[4:]) % 4])
     d = gapped_inputs(cfg)
     g = {k: (None if v is None else v.cuda()) for k, v in d.items()}
     ig = Guarded((cfg.T, cfg.top_k), torch.int32)

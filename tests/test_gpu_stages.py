@@ -170,7 +170,8 @@ def _ffn_case(dtype, act, E, rows_per_expert, H, F, seed=11):
     (2, [300, 45], 512, 1376),             # F of the 32-expert workload (N tail 1376 % 256)
     (5, [512, 640, 383, 0, 129], 384, 512),   # even / odd m-tile counts per expert
 ])
-@pytest.mark.parametrize("variant", ["rows128", "rows256_pair", "tokens_pair"])
+@pytest.mark.parametrize("variant", ["rows128", "rows256_pair", "tokens_pair",
+                                     "tokens_pair_nosplit"])
 def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
     """Every kernel against the oracle, with R_max - R = 37 spare rows: the spare
     rows of x_perm hold NaN (a kernel that mixes rows would spread them), the
