@@ -49,8 +49,19 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,           /* ws smaller than moe_workspace_bytes()               */
   MOE_ERR_UNSUPPORTED = 4,         /* sizes outside the limits above                      */
   MOE_ERR_CUDA = 5,                /* a CUDA runtime or driver call failed                */
-  MOE_ERR_TIMEOUT = 6              /* a kernel's bounded pipeline wait ran out            */
+  MOE_ERR_TIMEOUT = 6,             /* a kernel's bounded pipeline wait ran out            */
+  MOE_ERR_BOUNDS = 7               /* debug build only: an internal index fell outside its
+                                      buffer; the access was skipped (see below)           */
 } moe_status;
+
+/* Debug build.  libmoe_b200_debug.so is the same library compiled with
+ * MOE_DEBUG: before the accesses they guard, kernels check internal indices
+ * (scatter destination rows, router expert ids, combine rows against the
+ * T x k rows of y, grouped-GEMM tiles against the output and the K-split
+ * areas); a failed check records MOE_ERR_BOUNDS in the status word and skips
+ * the access instead of trapping.  Results are otherwise identical.
+ * Logging.  With MOE_LOG=1 in the environment when the library loads, every
+ * call prints its launch plan (kernel, grid, tiles, splits) to stderr.      */
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
@@ -159,7 +170,10 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* row_token, const v
  * summed in slot order in fp32 and rounded once to dt; no atomics, so the
  * result is bit-identical from run to run.  topk_gate may be NULL: every
  * weight is 1, and with top_k = 1 the call is a plain row gather
- * out[t] = y[row_map[t,0]] (exact; zero where row_map is -1).               */
+ * out[t] = y[row_map[t,0]] (exact; zero where row_map is -1).  Every
+ * row_map entry must be -1 or a row of y: the call does not know y's row
+ * count and does not check (the debug build checks entries against T x k,
+ * the row count moe_permute produces, and skips the others).               */
 moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const int32_t* row_map,
                                  int T, int H, int top_k, moe_dtype dt, void* out,
                                  moe_stream_t stream);

@@ -4,6 +4,9 @@ Every function here checks tensor dtypes, devices, shapes and contiguity, turns
 tensors into raw pointers and calls the entry point of the same name on the
 current CUDA stream.  All arithmetic happens in the CUDA library; there is no
 fallback: importing this module raises if ``lib/libmoe_b200.so`` is missing.
+With ``MOE_LIBRARY=debug`` in the environment the module loads the debug build
+``lib/libmoe_b200_debug.so`` instead (device bounds checks that report
+MOE_ERR_BOUNDS; same results otherwise).
 
 Tensors are allocated with torch (PyTorch is used for device memory and streams
 only).  Expert ids are int32, as the MoE fused operators require (an int64
@@ -17,17 +20,18 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libmoe_b200.so")
+RELEASE_LIB_PATH = os.path.join(_PKG, "lib", "libmoe_b200.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "lib", "libmoe_b200_debug.so")
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("MOE_LIBRARY") == "debug" else RELEASE_LIB_PATH
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with `python -m routing_grouped_expert_moe_b200.build`")
 
-_lib = ctypes.CDLL(LIB_PATH)
 
 # status codes (moe_status)
 OK, ERR_INVALID_ARG, ERR_INDEX_OUT_OF_RANGE, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, \
-    ERR_TIMEOUT = range(7)
+    ERR_TIMEOUT, ERR_BOUNDS = range(8)
 F32, BF16 = 0, 1
 ACT = {"swiglu": 0, "gelu": 1, "identity": 2}
 
@@ -68,10 +72,19 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (ctypes.c_char_p, []),
 }
-for _name, (_res, _args) in _SIGS.items():
-    _fn = getattr(_lib, _name)
-    _fn.restype = _res
-    _fn.argtypes = _args
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Opens a build of the library and declares every entry point's signature."""
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library(LIB_PATH)
 
 EXPORTED = tuple(_SIGS)
 

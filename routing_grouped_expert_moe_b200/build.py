@@ -1,6 +1,9 @@
 """Build lib/libmoe_b200.so from csrc/*.cu with nvcc for sm_100a (in-tree).
 
-Usage: python -m routing_grouped_expert_moe_b200.build [--force] [--jobs N]
+Usage: python -m routing_grouped_expert_moe_b200.build [--force] [--jobs N] [--debug]
+
+--debug builds lib/libmoe_b200_debug.so instead: the same sources compiled with
+MOE_DEBUG, whose device bounds checks record MOE_ERR_BOUNDS and skip the access.
 """
 from __future__ import annotations
 
@@ -18,6 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 BUILDDIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(LIBDIR, "libmoe_b200.so")
+LIB_DEBUG = os.path.join(LIBDIR, "libmoe_b200_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -48,15 +52,18 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, jobs: int = 8, verbose: bool = False, extra=None) -> str:
+def build(force: bool = False, jobs: int = 8, verbose: bool = False, extra=None,
+          debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    objdir = os.path.join(BUILDDIR, "debug") if debug else BUILDDIR
     os.makedirs(LIBDIR, exist_ok=True)
-    os.makedirs(BUILDDIR, exist_ok=True)
+    os.makedirs(objdir, exist_ok=True)
     nvcc = _nvcc()
     srcs, hdrs = _sources(), _headers()
-    flags = NVCC_FLAGS + ARCH + list(extra or [])
+    flags = NVCC_FLAGS + ARCH + (["-DMOE_DEBUG"] if debug else []) + list(extra or [])
 
     def compile_one(src):
-        obj = os.path.join(BUILDDIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         if force or _stale(obj, [src] + hdrs):
             cmd = [nvcc, *flags, "-c", src, "-o", obj]
             if verbose:
@@ -70,13 +77,13 @@ def build(force: bool = False, jobs: int = 8, verbose: bool = False, extra=None)
 
     with ThreadPoolExecutor(max_workers=jobs) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or _stale(LIB, objs):
-        cmd = [nvcc, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart_static", "-ldl", "-lrt",
+    if force or _stale(lib, objs):
+        cmd = [nvcc, *ARCH, "-shared", "-o", lib, *objs, "-lcudart_static", "-ldl", "-lrt",
                "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 def main(argv=None):
@@ -85,10 +92,11 @@ def main(argv=None):
     ap.add_argument("--jobs", type=int, default=8)
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/spill usage")
+    ap.add_argument("--debug", action="store_true", help="build libmoe_b200_debug.so")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_v else None
     print(build(force=a.force or a.ptxas_v, jobs=a.jobs, verbose=a.verbose or a.ptxas_v,
-                extra=extra))
+                extra=extra, debug=a.debug))
 
 
 if __name__ == "__main__":

@@ -2,11 +2,15 @@
 // workspace layout and the launch sequence of each entry point.  No entry
 // point allocates device memory or synchronises the stream (except
 // moe_get_device_status, whose job is to synchronise).
+#include <cxxabi.h>
+
 #include <atomic>
 #include <climits>
-#include <cstdlib>
 #include <cmath>
+#include <cstdarg>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "kernels.h"
@@ -24,7 +28,7 @@ Tuning read_tuning() {
   Tuning t;
   t.pdl = env_int("MOE_PDL", 1) != 0;
   const int v = env_int("MOE_GEMM_VARIANT", 0);
-  t.gemm_variant = (v >= 1 && v <= 3) ? v : 0;
+  t.gemm_variant = (v >= 1 && v <= 4) ? v : 0;
   t.gemm_ctas = env_int("MOE_GEMM_CTAS", 0);
   t.epi_sleep_ns = env_int("MOE_EPI_SLEEP", t.epi_sleep_ns);
   if (t.epi_sleep_ns < 0) t.epi_sleep_ns = 0;
@@ -33,6 +37,7 @@ Tuning read_tuning() {
   t.tokn_nacc = env_int("MOE_TOKN_NACC", 0);
   t.tokn_bk = env_int("MOE_TOKN_BK", 0);
   t.tokn_split = env_int("MOE_TOKN_SPLIT", 2);
+  t.log = env_int("MOE_LOG", 0) != 0;
   return t;
 }
 // Initialised when the library is loaded.
@@ -41,6 +46,29 @@ std::atomic<int> g_gemm_variant{g_tuning.gemm_variant};
 }  // namespace
 const Tuning& tuning() { return g_tuning; }
 int gemm_variant() { return g_gemm_variant.load(std::memory_order_relaxed); }
+
+void log_line(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::fputs("[moe] ", stderr);
+  std::vfprintf(stderr, fmt, ap);
+  std::fputc('\n', stderr);
+  va_end(ap);
+}
+
+void log_launch(const void* kern, dim3 grid, dim3 block, size_t smem, int cluster_x) {
+  const char* name = nullptr;
+  if (cudaFuncGetName(&name, kern) != cudaSuccess || name == nullptr) name = "?";
+  int dm = 0;
+  char* readable = abi::__cxa_demangle(name, nullptr, nullptr, &dm);
+  const char* shown = (readable != nullptr && dm == 0) ? readable : name;
+  if (std::strncmp(shown, "void ", 5) == 0) shown += 5;  // a template's return type
+  const char* paren = std::strchr(shown, '(');  // drop the parameter list
+  const int len = paren ? static_cast<int>(paren - shown) : static_cast<int>(std::strlen(shown));
+  log_line("launch %.*s grid=%u block=%u smem=%zu cluster=%d pdl=%d", len, shown, grid.x, block.x,
+           smem, cluster_x, tuning().pdl ? 1 : 0);
+  std::free(readable);
+}
 }  // namespace moe
 
 namespace {
@@ -384,7 +412,7 @@ moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const in
   if (!y || !row_map || !out || !aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (!index_range_ok(T, top_k, H)) return MOE_ERR_UNSUPPORTED;
   return cuda_status(launch_combine(y, topk_gate, row_map, T, H, top_k, dt == MOE_BF16, out,
-                                    num_sms_current(), as_stream(stream)));
+                                    num_sms_current(), as_stream(stream), nullptr));
 }
 
 // ---------------------------------------------------------------- router statistics
@@ -521,7 +549,7 @@ moe_status moe_expert_matmul(const void* x, const void* expert_weight,
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   // back to token order: out[t] = y[row_map[t]] (weight 1)
   return cuda_status(launch_combine(y, nullptr, row_map, T, I, 1, dt == MOE_BF16, out,
-                                    num_sms_current(), s));
+                                    num_sms_current(), s, status));
 }
 
 }  // extern "C"
@@ -650,7 +678,7 @@ moe_status forward_impl(const void* x, const void* w_gate, const float* gate_bia
   if (st != MOE_OK) return st;
   if (mark(5) != cudaSuccess) return MOE_ERR_CUDA;
   // 4. combine
-  if (launch_combine(y, topk_gate, row_map, T, H, top_k, bf16, out, nsm, s) != cudaSuccess)
+  if (launch_combine(y, topk_gate, row_map, T, H, top_k, bf16, out, nsm, s, status) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(mark(6));
 }
@@ -888,6 +916,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_BOUNDS: return "MOE_ERR_BOUNDS";
   }
   return "MOE_ERR_UNKNOWN";
 }

@@ -68,7 +68,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kCombineThreads)
     k_combine(const uint8_t* __restrict__ y, const float* __restrict__ gate,
               const int32_t* __restrict__ row_map, int T, int H, int k, int split,
-              uint8_t* __restrict__ out) {
+              uint8_t* __restrict__ out, int* status) {
   pdl_wait_and_trigger();
   constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
   constexpr int EB = BF16 ? 2 : 4;
@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
     for (int s = 0; s < kMaxTopK; ++s) {
       rows[s] = s < k ? __ldg(row_map + static_cast<size_t>(t) * k + s) : -1;
+      // y has the T x k rows of the permute's layout
+      if (rows[s] >= 0 && !MOE_DCHECK(rows[s] < T * k, status)) rows[s] = -1;
       g[s] = s < k ? (gate ? __ldg(gate + static_cast<size_t>(t) * k + s) : 1.f) : 0.f;
     }
     // two 16-byte vectors per lane and round: every load of both is in flight
@@ -112,7 +114,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 }
 
 cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
-                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s) {
+                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s,
+                           int* status) {
   const int warps_per_cta = kCombineThreads / 32;
   // split a row over several warps when the tokens alone leave the GPU short
   // of warps (about 32 per SM keep enough loads in flight)
@@ -125,13 +128,15 @@ cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_
   const long long cap = static_cast<long long>(num_sms) * 8;  // resident CTAs; more loop inside
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
+  if (log_enabled())
+    log_line("combine T=%d H=%d k=%d: %d warp(s) per token row, %lld CTAs", T, H, k, split, grid);
   if (dt_bf16)
     return launch_kernel(k_combine<true>, dim3(static_cast<unsigned>(grid)), dim3(kCombineThreads),
                          0, s, 1, static_cast<const uint8_t*>(y), gate, row_map, T, H, k, split,
-                         static_cast<uint8_t*>(out));
+                         static_cast<uint8_t*>(out), status);
   return launch_kernel(k_combine<false>, dim3(static_cast<unsigned>(grid)), dim3(kCombineThreads),
                        0, s, 1, static_cast<const uint8_t*>(y), gate, row_map, T, H, k, split,
-                       static_cast<uint8_t*>(out));
+                       static_cast<uint8_t*>(out), status);
 }
 
 }  // namespace moe

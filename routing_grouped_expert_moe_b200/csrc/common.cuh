@@ -25,6 +25,17 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);  // the first error wins
 }
 
+// Debug builds (compiled with MOE_DEBUG) check internal indices before the
+// accesses they guard: a failed check records MOE_ERR_BOUNDS and the caller
+// skips the access.  Release builds compile every check to `true`.
+constexpr int kStatusBounds = 7;
+#ifdef MOE_DEBUG
+#define MOE_DCHECK(cond, status) \
+  ((cond) || (::moe::record_status((status), ::moe::kStatusBounds), false))
+#else
+#define MOE_DCHECK(cond, status) (true)
+#endif
+
 // Programmatic dependent launch: wait until the grid this one depends on has
 // completed (no-op without such a dependency), then let the next grid in the
 // stream be scheduled (its own wait keeps it from reading this grid's output

@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * G_ACC_N);
-      const bool row_ok = row < ti.rows;
+      const bool row_ok = row < ti.rows && MOE_DCHECK(ti.m0 + row < args.R_max, args.status);
       const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;
@@ -304,6 +304,12 @@ cudaError_t launch_gemm_tc(int mode, bool gather, const void* a_src, int a_rows,
   const int cap = tuning().gemm_ctas;
   if (cap >= 2 && cap < num_sms) num_sms = cap;
   const int variant = choose_variant(mode, gather, g, num_sms);
+  if (log_enabled())
+    log_line("grouped GEMM mode=%d (%s) gather=%d rows<=%d N=%d K=%d E=%d: %s", mode,
+             mode == 1 ? "SwiGLU" : (mode == 0 ? "GELU" : "down"), gather ? 1 : 0, g.R_max, g.N,
+             g.K, g.E,
+             variant == 3 ? "token-as-N pair tiles"
+                          : (variant == 2 ? "256-row pair tiles" : "128-row tiles"));
   if (variant == 3 && g.sched != nullptr)
     return launch_gemm_tokn(mode, a_src, a_rows, b1, b3, ga, num_sms, s);
   CUtensorMap ma, mb1, mb3, mo;

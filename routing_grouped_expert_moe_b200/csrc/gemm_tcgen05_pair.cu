@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * G_ACC_N);
-      const bool row_ok = row < ti.rows;
+      const bool row_ok = row < ti.rows && MOE_DCHECK(ti.m0 + row < args.R_max, args.status);
       const bool box_full = q * 32 + 32 <= ti.rows;  // all 32 rows of this warp in the tile
       __nv_bfloat16* orow =
           row_ok ? out + static_cast<size_t>(ti.m0 + row) * args.N + ti.n0 : nullptr;

@@ -504,8 +504,12 @@ __global__ void __launch_bounds__(TokCfg<MODE, NACC, BK>::THREADS, 1)
       // [chunk / 2][acc][token / 4][lane][token % 4], so that a warp moves 512
       // contiguous bytes per float4 access.
       const size_t wslot = static_cast<size_t>((static_cast<int>(rank) * 8 + (warp - 2)) * 4 * 2 * 1024);
-      bool emit = true;
-      if (ti.unit >= 0) {
+      // the tile inside the output and, for a K-split part, inside the split areas
+      bool emit = MOE_DCHECK(ti.row0 >= 0 && ti.row0 + ti.rows <= args.R_max && ti.col0 < args.N &&
+                                 (ti.unit < 0 || (ti.unit < args.split_units &&
+                                                  ti.stile < args.split_tiles)),
+                             args.status);
+      if (ti.unit >= 0 && emit) {
         float* mine = args.split_ws + static_cast<size_t>(ti.unit) * kSplitUnitFloats + wslot;
 #pragma unroll 1
         for (int c = half; c < nch; c += 2) {
@@ -608,6 +612,10 @@ static cudaError_t launch_tokn_t(const CUtensorMap* x, const CUtensorMap& w1,
                                  int num_sms, cudaStream_t s) {
   using C = TokCfg<MODE, NACC, BK>;
   auto kern = k_gemm_tokn<MODE, NACC, BK>;
+  if (log_enabled())
+    log_line("token-as-N GEMM: %d accumulator(s) per tile, K %d per stage, %d stages of %d KB, "
+             "%d producer warps, K-split tail %s", NACC, BK, C::STAGES, C::STAGE_BYTES / 1024,
+             C::PROD, g.split_max > 1 && g.split_ws != nullptr ? "allowed" : "off");
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   return launch_kernel(kern, dim3((num_sms / 2) * 2), dim3(C::THREADS), C::SMEM, s, 2, x[0], x[1],

@@ -23,6 +23,7 @@ struct Tuning {
   int tokn_nacc = 0;            // MOE_TOKN_NACC=1|2: force the accumulators per tile (GELU, down)
   int tokn_bk = 0;              // MOE_TOKN_BK=64|128: force the K per pipeline stage
   int tokn_split = 2;           // MOE_TOKN_SPLIT=1: no K-split of the last partial wave
+  bool log = false;             // MOE_LOG=1: print launch plans to stderr
 };
 const Tuning& tuning();
 // Grouped-GEMM kernel choice: 0 automatic, 1 | 2 | 3 forced (moe_set_gemm_variant;
@@ -36,6 +37,13 @@ int gemm_variant();
 // it touches global memory, which returns once the predecessor grid has
 // completed and its writes are visible.
 inline bool pdl_enabled() { return tuning().pdl; }
+
+// MOE_LOG=1 (read when the library loads): launch plans on stderr, one line
+// per launch (kernel, grid, block, shared memory, cluster) and one per plan
+// decision (router split, GEMM variant and tile shape, scatter/combine split).
+inline bool log_enabled() { return tuning().log; }
+void log_line(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+void log_launch(const void* kern, dim3 grid, dim3 block, size_t smem, int cluster_x);
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -61,6 +69,7 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
+  if (log_enabled()) log_launch(reinterpret_cast<const void*>(kern), grid, block, smem, cluster_x);
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
@@ -165,8 +174,10 @@ cudaError_t launch_copy_rows(const void* a_src, const GemmArgs& g, int elem_byte
                              cudaStream_t s);
 
 // ---------------------------------------------------------------- combine
+// status (nullable): where a debug build records a row_map entry outside y.
 cudaError_t launch_combine(const void* y, const float* gate, const int32_t* row_map, int T,
-                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s);
+                           int H, int k, int dt_bf16, void* out, int num_sms, cudaStream_t s,
+                           int* status);
 
 // ---------------------------------------------------------------- router statistics
 // Per-expert pre-drop counts (summed from the router's per-tile histogram) and

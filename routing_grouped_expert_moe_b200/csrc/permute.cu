@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kPermThreads) k_scatter(PermuteArgs a) {
       int row = -1;
       if (e >= 0) {
         const int rank = base_s[e] + wcnt[warp][e] + rank_w;
-        if (rank < a.cap) {
+        if (rank < a.cap && MOE_DCHECK(off_s[e] + rank < a.T * a.k, a.status)) {
           row = off_s[e] + rank;
           if (part == 0) a.row_token[row] = i / a.k;
         }
@@ -198,6 +198,10 @@ cudaError_t launch_hist(const PermuteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_scatter(const PermuteArgs& a, cudaStream_t s) {
   if (a.BT * a.k > kScatterMaxPairs) return cudaErrorInvalidValue;
+  if (log_enabled())
+    log_line("scatter T=%d k=%d E=%d: %d token tiles of %d, %d CTAs per tile, capacity %d%s", a.T,
+             a.k, a.E, a.tiles, a.BT, a.split > 0 ? a.split : 1, a.cap,
+             a.x_perm ? ", rows copied to x_perm" : "");
   return launch_kernel(k_scatter, dim3(a.tiles * (a.split > 0 ? a.split : 1)), dim3(kPermThreads),
                        0, s, 1, a);
 }

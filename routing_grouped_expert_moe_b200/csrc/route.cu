@@ -91,7 +91,8 @@ __device__ void route_select_and_count(const float* logits_s, int ls_stride, int
   const int n = BT * k;
   for (int base = warp * 32; base < n; base += nwarps * 32) {
     const int i = base + lane;
-    const int e = i < n ? sel_s[i] : -1;
+    int e = i < n ? sel_s[i] : -1;
+    if (e >= 0 && !MOE_DCHECK(e < E, a.status)) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt_s[e], __popc(peers));
   }
@@ -204,6 +205,10 @@ RoutePlan route_plan(int T, int H, int E, int dt_bf16, int num_sms, bool can_spl
 }
 
 cudaError_t launch_route(const RouteArgs& a, const RoutePlan& p, cudaStream_t s) {
+  if (log_enabled())
+    log_line("router T=%d H=%d E=%d k=%d: %s, %d token tiles of %d, H split over %d CTAs%s", a.T,
+             a.H, a.E, a.top_k, p.kind == 2 ? "tensor cores" : "CUDA cores", p.tiles, p.BT,
+             p.kind == 2 ? p.ck : 1, p.kind == 2 ? ", experts padded to the MMA's N" : "");
   if (p.kind == 2) return launch_route_tc(a, p, s);
   const size_t smem = (kSimtBT * a.E + kSimtBT * 8 + 256) * 4;
   if (a.dt_bf16)

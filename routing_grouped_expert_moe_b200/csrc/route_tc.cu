@@ -92,7 +92,7 @@ __device__ __forceinline__ void route_tc_finish(const RouteArgs& a, int tile, in
       if (s < a.top_k) { z[s] = expf(key_value(best[s]) - l0); sum += z[s]; }
 #pragma unroll
     for (int s = 0; s < K; ++s)
-      if (s < a.top_k) {
+      if (s < a.top_k && MOE_DCHECK(key_expert(best[s]) < a.E, a.status)) {
         a.topk_idx[static_cast<size_t>(t) * a.top_k + s] = key_expert(best[s]);
         a.topk_gate[static_cast<size_t>(t) * a.top_k + s] = z[s] / sum;
       }

@@ -31,10 +31,24 @@ def test_header_functions_are_exported():
     assert set(names) == set(B.EXPORTED)
 
 
+def test_debug_build_exports_the_same_functions():
+    """libmoe_b200_debug.so (MOE_DEBUG device bounds checks) is a drop-in
+    replacement: same entry points, same host-side argument checks."""
+    assert os.path.exists(B.DEBUG_LIB_PATH), "build with `python -m routing_grouped_expert_moe_b200.build --debug`"
+    dbg = B.load_library(B.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    assert dbg.moe_status_string(B.ERR_BOUNDS) == b"MOE_ERR_BOUNDS"
+    # host-side rejection before any CUDA call, as in the release build
+    assert dbg.moe_route(None, None, None, 4, 64, 8, 9, B.BF16, None, None, None, None) == \
+        B.ERR_INVALID_ARG
+
+
 def test_status_strings_and_version():
     assert B.status_string(B.OK) == "MOE_OK"
     assert B.status_string(B.ERR_INDEX_OUT_OF_RANGE) == "MOE_ERR_INDEX_OUT_OF_RANGE"
     assert B.status_string(B.ERR_TIMEOUT) == "MOE_ERR_TIMEOUT"
+    assert B.status_string(B.ERR_BOUNDS) == "MOE_ERR_BOUNDS"
     assert "sm_100a" in B.version()
 
 
