@@ -24,8 +24,9 @@ single-device forward of those tokens over all E experts gives:
      slot its input came from, and the local combine sums the gated rows.
 
 Rows travel as raw bytes, so any storage type crosses unchanged.  The split
-sizes are read on the host (one device-to-host read of the offsets, one of
-the received counts): all-to-all with uneven splits needs them there.
+sizes are read on the host, since all-to-all with uneven splits takes them
+there: the count exchange runs on the device first, so one device-to-host
+read per forward brings back this rank's offsets and the counts it receives.
 
 The per-rank compute steps are the C ABI's kernels (`CudaSteps`); torch.distributed
 (NCCL between GPUs) carries the two exchanges.
@@ -201,19 +202,22 @@ def ep_forward(x, w_gate, gate_bias, w1_local, w3_local, w2_local, top_k: int,
     if T > 0:
         idx, gate = steps.route(x, w_gate, gate_bias, top_k)
         x_perm, offsets_d, row_map = steps.permute(x, idx, E, capacity_factor)
-        offsets = steps.to_host(offsets_d).astype(np.int64)
     else:
         gate = row_map = None
         x_perm = x.new_empty(0, H)
-        offsets = np.zeros(E + 1, dtype=np.int64)
+        offsets_d = torch.zeros(E + 1, dtype=torch.int32, device=dev)
+
+    # 2. kept-row counts per (destination, expert), exchanged on the device; then
+    # the forward's one host read brings back this rank's offsets and the counts
+    # it receives together (an uneven all-to-all takes its split sizes on the host)
+    offsets_d = offsets_d.to(torch.int32)
+    kept_d = offsets_d[1:] - offsets_d[:-1]
+    recv_kept_d = torch.empty(E, dtype=torch.int32, device=dev)
+    dist.all_to_all_single(recv_kept_d, kept_d, group=group)
+    both = steps.to_host(torch.cat([offsets_d, recv_kept_d])).astype(np.int64)
+    offsets, recv_kept = both[:E + 1], both[E + 1:].reshape(G, el)
     send = split_rows(offsets, G)
     R = int(offsets[E])
-
-    # 2. kept-row counts per (destination, expert)
-    kept = torch.from_numpy(np.diff(offsets).astype(np.int32)).to(dev)
-    recv_kept_d = torch.empty(E, dtype=torch.int32, device=dev)
-    dist.all_to_all_single(recv_kept_d, kept, group=group)
-    recv_kept = steps.to_host(recv_kept_d).astype(np.int64).reshape(G, el)
     recv = recv_kept.sum(axis=1)
     R_in = int(recv.sum())
 

@@ -46,6 +46,7 @@ class OracleSteps:
 
     def __init__(self, dtype: str):
         self.dtype = dtype
+        self.host_reads = 0
 
     def _store(self, a, like):
         return torch.from_numpy(np.asarray(a, dtype=np.float64)).to(like.dtype)
@@ -83,6 +84,7 @@ class OracleSteps:
         return self._store(O.combine(as_np(y), gate.numpy(), row_map.numpy(), self.dtype), y)
 
     def to_host(self, t):
+        self.host_reads += 1
         return t.numpy()
 
     def from_host(self, a, like):
@@ -135,10 +137,14 @@ def _rank_main(rank: int, world: int, port: int, names, q):
             E, el = d["E"], d["E"] // world
             sl = slice(rank * el, (rank + 1) * el)
             local = lambda w: None if w is None else w[sl].contiguous()  # noqa: E731
-            outs = [EP.ep_forward(d["x"], d["w_gate"], d["gate_bias"], local(d["w1"]),
-                                  local(d["w3"]), local(d["w2"]), d["k"], d["cf"], d["act"], E,
-                                  steps=OracleSteps(d["dtype"]), overlap=ov)
-                    for ov in (False, True)]
+            outs = []
+            for ov in (False, True):
+                steps = OracleSteps(d["dtype"])
+                outs.append(EP.ep_forward(d["x"], d["w_gate"], d["gate_bias"], local(d["w1"]),
+                                          local(d["w3"]), local(d["w2"]), d["k"], d["cf"],
+                                          d["act"], E, steps=steps, overlap=ov))
+                # split sizes reach the host once per forward
+                assert steps.host_reads == 1, (name, ov, steps.host_reads)
             for out in outs:
                 assert out.shape == d["x"].shape and out.dtype == d["x"].dtype
             # the overlapped exchange moves the same rows: the same bits
