@@ -634,11 +634,6 @@ cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void
                              const void* b3, const GemmArgs& g_in, int num_sms, cudaStream_t s) {
   if (g_in.sched == nullptr) return cudaErrorInvalidValue;
   GemmArgs g = g_in;
-  // K-split tail: measured on the Mixtral-shaped, 128-expert and 32-expert
-  // layers, the SwiGLU GEMM-1 (one accumulator pair, epilogue not overlapped)
-  // gains 1-2.5%; the GELU and down-projection GEMMs (double-buffered) lose
-  // up to 1%, so they keep whole tiles.
-  g.split_max = (mode == 1 && gemm_variant() != 4) ? tuning().tokn_split : 1;
   // Tile shape per GEMM (measured on the Mixtral-shaped and page-1 layers):
   // SwiGLU keeps two accumulators (W1, W3) and 4 stages of K = 64; GELU one
   // double-buffered accumulator and 3 stages of K = 128; the down-projection
@@ -647,9 +642,15 @@ cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void
   bool two = mode == 1;
   if (mode == 2)
     two = static_cast<double>(g.R_max) * g.K * 2.0 > 64.0 * 1024 * 1024;
-  int bk = two ? 64 : 128;
   if (mode != 1 && tuning().tokn_nacc != 0) two = tuning().tokn_nacc == 2;
+  int bk = two ? 64 : 128;
   if (tuning().tokn_bk != 0) bk = tuning().tokn_bk == 64 ? 64 : 128;
+  // K-split tail: measured on the Mixtral-shaped, 128-expert and 32-expert
+  // layers, the SwiGLU GEMM-1 (W1 and W3 accumulators fill TMEM, epilogue not
+  // overlapped) gains 1-2.5%; the down-projection loses up to 1% (two
+  // accumulators: page-1 and 32-expert layers) or gains nothing, and the
+  // double-buffered GELU GEMM-1 gains nothing, so they keep whole tiles.
+  g.split_max = (mode == 1 && gemm_variant() != 4) ? tuning().tokn_split : 1;
   CUtensorMap mx[3], mw1, mw3, mo;
   const uint32_t box_rows[3] = {32, 64, 128};
   for (int i = 0; i < 3; ++i)
