@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the grouped GEMM kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source they were taken on; None until captured.
-NCU_TRAFFIC = {"source_sha": "dba4732d11818b55", "workload": "mixtral_e8",
-               "bytes_per_forward": 2.9999e9}
+NCU_TRAFFIC = {"source_sha": "b5e2d7fd53de478b", "workload": "mixtral_e8",
+               "bytes_per_forward": 2.9972e9}
 
 
 def parse_args(argv=None):
@@ -430,7 +430,7 @@ def _run_ep_one_rank(args, B, dev, flush, steps, warmup) -> int:
                        "parallelism": "ep1 (one NCCL rank: every exchange is a local copy)"},
             "fused_forward_ms": f_ms, "ep_ms": e_ms, "ep_overlap_ms": o_ms,
             "note": "CUDA events around each call on the current stream; the expert-parallel "
-                    "path reads its split sizes on the host twice per forward, and the GPU "
+                    "path reads its split sizes on the host once per forward, and the GPU "
                     "idles meanwhile"}
     print(json.dumps(line), flush=True)
     return 0
@@ -584,6 +584,11 @@ def main(argv=None):
         dist.barrier()
     clocks = sampler.stop(t_wall0, t_wall1)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    q = sorted(step_ms)
+    n10 = max(1, len(step_ms) // 10)
+    step_stats = {"p10": q[len(q) // 10], "p50": q[len(q) // 2], "p90": q[(9 * len(q)) // 10],
+                  "first_tenth_mean": statistics.mean(step_ms[:n10]),
+                  "last_tenth_mean": statistics.mean(step_ms[-n10:])}
     total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(T, world, args.steps, total_ms)
@@ -688,6 +693,7 @@ def main(argv=None):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "step_ms_stats": step_stats,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": cfg.dtype, "data": "synthetic (seeded Philox normal inputs, random-init weights)",
         "config": {**workload_desc(cfg),

@@ -38,6 +38,7 @@ Tuning read_tuning() {
   t.tokn_bk = env_int("MOE_TOKN_BK", 0);
   t.tokn_split = env_int("MOE_TOKN_SPLIT", 2);
   t.log = env_int("MOE_LOG", 0) != 0;
+  t.tokn_stash = env_int("MOE_TOKN_STASH", 1) != 0;
   return t;
 }
 // Initialised when the library is loaded.

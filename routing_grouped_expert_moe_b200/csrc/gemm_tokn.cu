@@ -723,7 +723,9 @@ cudaError_t launch_gemm_tokn(int mode, const void* a_src, int a_rows, const void
   switch (mode) {
     case 0: return two ? launch_tokn_bk<0, 2>(bk, mx, mw1, mw3, mo, g, num_sms, s)
                        : launch_tokn_bk<0, 1>(bk, mx, mw1, mw3, mo, g, num_sms, s);
-    case 1: return launch_tokn_bk<1, 2, true>(bk, mx, mw1, mw3, mo, g, num_sms, s);
+    case 1: return tuning().tokn_stash
+                       ? launch_tokn_bk<1, 2, true>(bk, mx, mw1, mw3, mo, g, num_sms, s)
+                       : launch_tokn_bk<1, 2, false>(bk, mx, mw1, mw3, mo, g, num_sms, s);
     case 2: return two ? launch_tokn_bk<2, 2>(bk, mx, mw1, mw3, mo, g, num_sms, s)
                        : launch_tokn_bk<2, 1>(bk, mx, mw1, mw3, mo, g, num_sms, s);
   }

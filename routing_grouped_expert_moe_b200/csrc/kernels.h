@@ -24,6 +24,7 @@ struct Tuning {
   int tokn_bk = 0;              // MOE_TOKN_BK=64|128: force the K per pipeline stage
   int tokn_split = 2;           // MOE_TOKN_SPLIT=1: no K-split of the last partial wave
   bool log = false;             // MOE_LOG=1: print launch plans to stderr
+  bool tokn_stash = true;       // MOE_TOKN_STASH=0: SwiGLU epilogue holds TMEM while storing
 };
 const Tuning& tuning();
 // Grouped-GEMM kernel choice: 0 automatic, 1 | 2 | 3 forced (moe_set_gemm_variant;
