@@ -10,11 +10,15 @@
 // ceil(n / 16) * 16 token columns instead of a whole 128- or 256-row tile; a
 // segment of more than 256 rows is split into equal groups of at most 256.
 //
-// Operand bytes per MMA clock decide this kernel's speed: one SM takes about
-// 55 bytes per clock from TMA.  A pair tile of 256 weight columns x 256 tokens
-// x 64 K moves 16 KB of weights and 16 KB of tokens into each SM per 512 MMA
-// clocks (64 B/clk); the SwiGLU form keeps two accumulators (W1 and W3) over
-// the same token tile, 48 KB per 1024 clocks (48 B/clk).
+// The operand stream into each SM paces this kernel.  A pair tile of 256
+// weight columns x 256 tokens x 64 K moves 16 KB of weights and 16 KB of
+// tokens into each SM per 512 MMA clocks (64 B/clk); the SwiGLU form keeps two
+// accumulators (W1 and W3) over the same token tile, 48 KB per 1024 clocks
+// (48 B/clk).  Measured with every SM streaming, a pipeline stage takes about
+// the same time whatever the tile's token count (the loads' latency under
+// load, with 192 KB of stages in flight per SM, paces the ring), so a full
+// 256-token tile keeps the tensor pipe ~91% busy over its main loop and a
+// smaller token group leaves the rest idle.
 //
 // NACC accumulators per tile: NACC = 1 double-buffers one 256-column
 // accumulator so the epilogue of a tile overlaps the next tile's main loop;
@@ -25,12 +29,12 @@
 // one launch take about the same time and the last wave, total mod the CTA
 // pairs, runs on a fraction of the GPU.  When at most half the pairs are
 // left for it (and the host asks for it: the SwiGLU GEMM-1), those last
-// tiles are cut along K into two parts.  Each part
-// writes its fp32 accumulators to the workspace, then counts itself in on a
-// ticket per epilogue warp; the part that comes second adds the other's sums
-// to its own (fp32 addition of two terms is commutative, so the result does
-// not depend on which part finished first) and runs the activation and the
-// stores.  No part waits for another.
+// tiles are cut along K into two parts.  Each part writes its fp32
+// accumulators to the workspace, then counts itself in on a ticket per
+// epilogue warp; the part that comes second adds the other's sums to its own
+// (fp32 addition of two terms is commutative, so the result does not depend
+// on which part finished first) and runs the activation and the stores.  No
+// part waits for another.
 //
 // Tiles are taken from a global counter (dynamic schedule: token groups of
 // different sizes take different times).  The first CTA's producer takes the
