@@ -179,7 +179,7 @@ def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
     that must survive."""
     if dtype == "f32" and variant != "rows128":
         pytest.skip("the fp32 path has a single CUDA-core kernel")
-    if gather and variant == "tokens_pair":
+    if gather and variant.startswith("tokens_pair"):
         pytest.skip("gathered rows always use the row-tiled kernels")
     gemm_variant(variant)
     E, rows, H, F = shape
@@ -211,6 +211,38 @@ def test_grouped_ffn(dtype, act, gather, shape, variant, gemm_variant):
     y.check("y")
     y.untouched(R * H * esz, R_max * H * esz, "y rows past R")
     ws.check("workspace")
+
+
+def test_grouped_ffn_ksplit_tail(gemm_variant):
+    """With room in the workspace the SwiGLU GEMM-1 cuts its last partial wave of
+    tiles in two along K: here 3 token groups x 2 output-column blocks = 6 tiles,
+    all of them in that wave, so all are split.  Against the oracle; bit-identical
+    on a second run (a sum of two fp32 parts does not depend on which part
+    finished first); within tolerance of the unsplit kernel, and different from it
+    in some element (the split's summation order ran); sentinels around y and the
+    workspace, split sums and tickets included."""
+    E, rows, H, F = 3, [256, 200, 77], 2048, 512
+    dt, x, w1, w3, w2, perm = _ffn_case("bf16", "swiglu", E, rows, H, F, seed=23)
+    ref = O.grouped_ffn(as_np(x), perm, as_np(w1), as_np(w3), as_np(w2), "swiglu", "bf16", E)
+    R = perm["R"]
+    offs = torch.from_numpy(perm["offsets"].astype(np.int32)).cuda()
+    x_perm = x[torch.from_numpy(perm["row_token"])].contiguous().cuda()
+    nbytes = B()._lib.moe_grouped_ffn_workspace_bytes(R, H, F, B().ACT["swiglu"], B().BF16, 0)
+    outs = []
+    for variant in ("tokens_pair", "tokens_pair", "tokens_pair_nosplit"):
+        gemm_variant(variant)
+        ws = guarded_workspace(nbytes)
+        y = Guarded((R, H), dt)
+        B().grouped_ffn(offs, w1.cuda(), w3.cuda(), w2.cuda(), "swiglu", x_perm=x_perm, ws=ws.t,
+                        y=y.t)
+        assert B().device_status(ws.t) == B().OK
+        y.check("y")
+        ws.check("workspace")
+        outs.append(y.t.clone())
+    for o in outs:
+        assert rel_err(as_np(o), ref) <= TOL["bf16"]
+    assert torch.equal(outs[0], outs[1])
+    assert not torch.equal(outs[0], outs[2])
 
 
 @pytest.mark.parametrize("act", ["swiglu", "gelu"])
