@@ -57,13 +57,15 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["layer", "expert_matmul", "route_stats", "ep_one_rank"],
+    ap.add_argument("--op", choices=["layer", "expert_matmul", "route_stats", "ep", "ep_one_rank"],
                     default="layer",
                     help="layer: the MoE layer (default, the headline); expert_matmul: the k=1\n"
                          "up-projection op on x[1024,4096] x W[8,4096,14336]; route_stats: the\n"
                          "router with its load statistics on the e32_long router shape;\n"
-                         "ep_one_rank: the expert-parallel forward on one NCCL rank (its\n"
-                         "exchanges and host reads) against the fused forward, --config workload")
+                         "ep: the expert-parallel forward, one rank per GPU (torchrun), each\n"
+                         "rank owning E/N experts and its own tokens of the --config workload\n"
+                         "(on one GPU also timed against the fused forward); ep_one_rank: the\n"
+                         "same as ep on one GPU")
     ap.add_argument("--hbm-copy-sweep", action="store_true",
                     help="time plain device copies at the memory stages' sizes and exit")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -400,38 +402,82 @@ def _time_steps(fn, steps: int, warmup: int, flush) -> list:
     return [a.elapsed_time(b) for a, b in ms]
 
 
-def _run_ep_one_rank(args, B, dev, flush, steps, warmup) -> int:
-    """The expert-parallel forward on a one-rank NCCL group: what its exchanges (here
-    local), host reads of the split sizes and regroup cost against the fused forward."""
+def _run_ep(args, B, flush, steps, warmup) -> int:
+    """The expert-parallel forward (expert_parallel.ep_forward), one rank per GPU:
+    rank r of N owns experts [r*E/N, (r+1)*E/N) and routes its own tokens; every
+    step is timed with CUDA events between barriers, and the job's time per step
+    is the slowest rank's.  On one rank every exchange is a local copy, and the
+    fused forward is timed beside it for the cost of the exchanges' host reads,
+    the regroup and the separate launches."""
     import torch.distributed as tdist
     from routing_grouped_expert_moe_b200 import expert_parallel as EP
-    cfg = resolve_config(args.config, args.tokens)
-    d = synth.make_inputs(cfg)
-    g = {k: (None if v is None else v.to(dev)) for k, v in d.items()}
-    ws = B.alloc_workspace(B.workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k, cfg.act,
-                                             cfg.torch_dtype), dev)
-    out = torch.empty(cfg.T, cfg.H, dtype=cfg.torch_dtype, device=dev)
-    args_l = (g["x"], g["w_gate"], g["gate_bias"], g["w1"], g["w3"], g["w2"], cfg.top_k,
-              cfg.capacity_factor, cfg.act)
-    tdist.init_process_group("nccl", store=tdist.HashStore(), rank=0, world_size=1)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if world > 1:
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    else:
+        tdist.init_process_group("nccl", store=tdist.HashStore(), rank=0, world_size=1)
     try:
-        fused = _time_steps(lambda: B.forward(*args_l, out=out, ws=ws), steps, warmup, flush)
-        ep = _time_steps(lambda: EP.ep_forward(*args_l, cfg.E), steps, warmup, flush)
-        ep_ov = _time_steps(lambda: EP.ep_forward(*args_l, cfg.E, overlap=True), steps, warmup,
-                            flush)
+        cfg = resolve_config(args.config, args.tokens)
+        if cfg.E % world:
+            if rank == 0:
+                print(json.dumps({"metric": "expert-parallel layer tokens/s", "unavailable":
+                                  f"{cfg.E} experts do not split over {world} ranks"}), flush=True)
+            return 0
+        el = cfg.E // world
+        d = rank_inputs(cfg, rank)
+        sl = slice(rank * el, (rank + 1) * el)
+        local = lambda w: None if w is None else w[sl].contiguous().to(dev)  # noqa: E731
+        x, wg = d["x"].to(dev), d["w_gate"].to(dev)
+        b = None if d["gate_bias"] is None else d["gate_bias"].to(dev)
+        w1, w3, w2 = local(d["w1"]), local(d["w3"]), local(d["w2"])
+        ep_args = (x, wg, b, w1, w3, w2, cfg.top_k, cfg.capacity_factor, cfg.act, cfg.E)
+
+        def timed(fn):
+            for _ in range(warmup):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            tdist.barrier()
+            ms = []
+            for _ in range(steps):
+                flush.zero_()
+                s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s0.record()
+                fn()
+                s1.record()
+                ms.append((s0, s1))
+            torch.cuda.synchronize()
+            tdist.barrier()
+            mean_ms = statistics.mean(a.elapsed_time(z) for a, z in ms)
+            return max_over_ranks(mean_ms, tdist, dev)
+
+        e_ms = timed(lambda: EP.ep_forward(*ep_args))
+        o_ms = timed(lambda: EP.ep_forward(*ep_args, overlap=True))
+        f_ms = None
+        if world == 1:
+            ws = B.alloc_workspace(B.workspace_bytes(cfg.T, cfg.H, cfg.F, cfg.E, cfg.top_k,
+                                                     cfg.act, cfg.torch_dtype), dev)
+            out = torch.empty(cfg.T, cfg.H, dtype=cfg.torch_dtype, device=dev)
+            f_ms = timed(lambda: B.forward(x, wg, b, w1, w3, w2, cfg.top_k, cfg.capacity_factor,
+                                           cfg.act, out=out, ws=ws))
     finally:
         tdist.destroy_process_group()
-    f_ms, e_ms, o_ms = (statistics.mean(v) for v in (fused, ep, ep_ov))
-    line = {"metric": "expert-parallel layer tokens/s on one rank", "value": cfg.T / (e_ms / 1e3),
-            "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
-            "ms_per_step": e_ms, "higher_is_better": True, "dtype": cfg.dtype,
+    if rank != 0:
+        return 0
+    line = {"metric": "expert-parallel layer tokens/s", "value": cfg.T * world / (e_ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+            "ms_per_step": e_ms, "higher_is_better": True, "scaling": "weak", "dtype": cfg.dtype,
             "data": "synthetic (seeded Philox normal inputs, random-init weights)",
             "config": {**workload_desc(cfg), "l2": "flushed before every step",
-                       "parallelism": "ep1 (one NCCL rank: every exchange is a local copy)"},
-            "fused_forward_ms": f_ms, "ep_ms": e_ms, "ep_overlap_ms": o_ms,
-            "note": "CUDA events around each call on the current stream; the expert-parallel "
-                    "path reads its split sizes on the host once per forward, and the GPU "
-                    "idles meanwhile"}
+                       "parallelism": (f"ep{world} (rank r owns experts r*E/{world} .. "
+                                       f"(r+1)*E/{world}-1, every rank its own tokens)"
+                                       if world > 1 else
+                                       "ep1 (one NCCL rank: every exchange is a local copy)")},
+            "ep_ms": e_ms, "ep_overlap_ms": o_ms, "fused_forward_ms": f_ms,
+            "note": "CUDA events around each call on the current stream, slowest rank; the "
+                    "expert-parallel path reads its split sizes on the host once per forward"}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -439,13 +485,13 @@ def _run_ep_one_rank(args, B, dev, flush, steps, warmup) -> int:
 def run_op(args) -> int:
     """One JSON line for a single-op row (not the layer headline)."""
     from routing_grouped_expert_moe_b200 import binding as B
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     peaks, peak_src = load_peaks()
     steps, warmup = min(args.steps, 100), max(args.warmup, 3)
-    if args.op == "ep_one_rank":
-        return _run_ep_one_rank(args, B, dev, flush, steps, warmup)
+    if args.op in ("ep", "ep_one_rank"):
+        return _run_ep(args, B, flush, steps, warmup)
     if args.op == "expert_matmul":
         T, H, I, E, seed = 1024, 4096, 14336, 8, 5001
         x = synth.normal(seed, synth.STREAM_X, (T, H), 1.0, torch.bfloat16).to(dev)
