@@ -35,10 +35,12 @@ With overlap=True (and at least two experts per rank) the local experts form
 two groups, A = the first half and B = the rest, and the rows move as
 point-to-point messages per group, following the same pages' point that
 expert parallelism lets communication overlap computation: B's rows travel
-while A's experts run, and A's outputs travel back while B's experts run.  A
-group's rows for one destination are contiguous in the expert-ordered block
-(experts of a rank are consecutive), so every message is a slice of an
-existing buffer; a rank's rows for itself are copied locally.
+while A's experts run, and A's outputs travel back while B's experts run.
+Every (rank, local expert) block is a message of its own, a slice of the
+sender's expert-ordered rows, and lands at its place in an expert-major
+buffer (local expert, then source rank), so the group's rows go to the
+grouped FFN without a regroup and its outputs go back block by block; a
+rank's blocks for itself are copied locally.
 """
 from __future__ import annotations
 
@@ -102,13 +104,15 @@ def _bytes(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.uint8)
 
 
-def _post(sends, recvs, me, group, tag):
-    """Start one point-to-point round: sends[p] goes to rank p, recvs[p] is filled by
-    rank p (contiguous byte views, None when empty: both sides derive the same sizes
-    from the exchanged counts, so they skip the same messages).  The block for this
-    rank itself is copied locally.  Returns the pending requests."""
+def _post(msgs, me, group, tag):
+    """Start one point-to-point round.  msgs: (peer, send, recv) triples in an order
+    both sides of every pair derive alike from the exchanged counts (send: a
+    contiguous byte view going to the peer, recv: one the peer fills; None when
+    empty, so both sides skip the same messages).  Messages between two ranks
+    are matched in the order they are posted; a rank's blocks for itself are
+    copied locally.  Returns the pending requests."""
     ops = []
-    for peer, (snd, rcv) in enumerate(zip(sends, recvs)):
+    for peer, snd, rcv in msgs:
         if peer == me:
             if rcv is not None:
                 rcv.copy_(snd)
@@ -133,45 +137,55 @@ def _rows(buf, a, b):
 def _overlapped_experts(steps, x_perm, offsets, recv_kept, w1, w3, w2, act, G, el, me,
                         group, y_back):
     """Rows out, experts, rows back, in two expert groups that overlap (see the module
-    docstring); fills y_back (rows in the order of x_perm)."""
+    docstring); fills y_back (rows in the order of x_perm).  Each (rank, local
+    expert) block travels as a message of its own and lands in expert order
+    (local expert, then source rank), so the received rows go to the grouped FFN
+    as they are and its outputs go back block by block: no regroup."""
     H = x_perm.shape[1]
     halves = [(0, el // 2), (el // 2, el)]
-    recv_in = []                       # per group: its counts [G, group size], row starts
-    bufs = []                          # per group: the received rows
+    layouts = []                       # per group: block starts [group size, G], segment starts
+    bufs = []                          # per group: the received rows, expert-major
     pending = []
     keep = []                          # outputs still being sent back
     for gi, (j0, j1) in enumerate(halves):
-        rk = recv_kept[:, j0:j1]
-        cnt = rk.sum(axis=1)
-        starts = np.concatenate([[0], np.cumsum(cnt)])
+        rk = recv_kept[:, j0:j1]                       # [source, local expert of the group]
+        sizes = rk.T.reshape(-1)                       # expert-major: (j, s)
+        starts = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+        pos = starts[:-1].reshape(j1 - j0, G)
+        seg = np.concatenate([[0], np.cumsum(rk.sum(axis=0))]).astype(np.int64)
         buf = x_perm.new_empty(int(starts[-1]), H)
-        sends = [_rows(x_perm, int(offsets[d * el + j0]), int(offsets[d * el + j1]))
-                 for d in range(G)]
-        recvs = [_rows(buf, int(starts[s]), int(starts[s + 1])) for s in range(G)]
-        pending.append(_post(sends, recvs, me, group, tag=gi))
-        recv_in.append((rk, starts))
+        msgs = []
+        for p in range(G):             # per peer: its experts of the group, in order
+            for j in range(j0, j1):
+                a = int(pos[j - j0, p])
+                msgs.append((p, _rows(x_perm, int(offsets[p * el + j]),
+                                      int(offsets[p * el + j + 1])),
+                             _rows(buf, a, a + int(rk[p, j - j0]))))
+        pending.append(_post(msgs, me, group, tag=gi))
+        layouts.append((rk, pos, seg))
         bufs.append(buf)
-    back = []
     for gi, (j0, j1) in enumerate(halves):
         _wait(pending[gi])             # this group's rows are here; the next may still travel
-        rk, starts = recv_in[gi]
+        rk, pos, seg = layouts[gi]
         buf = bufs[gi]
         if buf.shape[0] > 0:
-            ids = steps.from_host(local_expert_ids(rk).reshape(-1, 1), buf)
-            x_loc, off_loc, map_loc = steps.permute(buf, ids, j1 - j0, 0.0)
             sl = slice(j0, j1)
-            y_loc = steps.grouped_ffn(x_loc, off_loc, None if w1 is None else w1[sl],
+            off = steps.from_host(seg.astype(np.int32), buf)
+            y_grp = steps.grouped_ffn(buf, off, None if w1 is None else w1[sl],
                                       None if w3 is None else w3[sl],
                                       None if w2 is None else w2[sl], act)
-            y_in = steps.unpermute(y_loc, map_loc)
         else:
-            y_in = buf
-        sends = [_rows(y_in, int(starts[s]), int(starts[s + 1])) for s in range(G)]
-        recvs = [_rows(y_back, int(offsets[d * el + j0]), int(offsets[d * el + j1]))
-                 for d in range(G)]
-        back.append(_post(sends, recvs, me, group, tag=2 + gi))
-        keep.append(y_in)
-    for w in back:
+            y_grp = buf
+        msgs = []
+        for p in range(G):
+            for j in range(j0, j1):
+                a = int(pos[j - j0, p])
+                msgs.append((p, _rows(y_grp, a, a + int(rk[p, j - j0])),
+                             _rows(y_back, int(offsets[p * el + j]),
+                                   int(offsets[p * el + j + 1]))))
+        pending.append(_post(msgs, me, group, tag=2 + gi))
+        keep.append(y_grp)
+    for w in pending[len(halves):]:
         _wait(w)
     del keep
 

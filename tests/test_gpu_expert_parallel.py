@@ -1,7 +1,8 @@
 """Expert-parallel forward on the GPU with one NCCL rank: every exchange runs
 (counts, rows out, rows back) through NCCL, and every compute step through the
-C ABI's kernels, including the k = 1 regroup and its inverse (the combine with
-no gates), in both the one-round and the two-group (overlapped) form.  More ranks need more GPUs than these tests get; the exchange logic
+C ABI's kernels: the one-round form with its k = 1 regroup and inverse (the
+combine with no gates), and the two-group (overlapped) form, whose per-expert
+blocks land in expert order.  More ranks need more GPUs than these tests get; the exchange logic
 over several ranks is checked on CPU ranks (test_expert_parallel.py)."""
 import numpy as np
 import pytest
