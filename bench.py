@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of the grouped GEMM kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source they were taken on; None until captured.
-NCU_TRAFFIC = {"source_sha": "5c203efbb20a8c8b", "workload": "mixtral_e8",
+NCU_TRAFFIC = {"source_sha": "82c78a976bf07d0f", "workload": "mixtral_e8",
                "bytes_per_forward": 2.9972e9}
 
 

@@ -15,10 +15,10 @@
 // tokens into each SM per 512 MMA clocks (64 B/clk); the SwiGLU form keeps two
 // accumulators (W1 and W3) over the same token tile, 48 KB per 1024 clocks
 // (48 B/clk).  Measured with every SM streaming, a pipeline stage takes about
-// the same time whatever the tile's token count (the loads' latency under
-// load, with 192 KB of stages in flight per SM, paces the ring), so a full
-// 256-token tile keeps the tensor pipe ~91% busy over its main loop and a
-// smaller token group leaves the rest idle.
+// the same time whatever the tile's token count (a fixed cost per stage plus
+// what one SM can bring in, ~47 B/clk), so a full 256-token SwiGLU tile keeps
+// the tensor pipe ~91% busy over its main loop and a smaller token group
+// leaves the rest idle.
 //
 // NACC accumulators per tile: NACC = 1 double-buffers one 256-column
 // accumulator so the epilogue of a tile overlaps the next tile's main loop;
