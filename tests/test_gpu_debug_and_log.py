@@ -120,3 +120,16 @@ def test_launch_plan_log():
                  "launch moe::k_gemm_tokn<1, 2"):
         assert part in text, (part, text)
     assert sum(ln.startswith("[moe] launch ") for ln in lines) == 6  # the fused forward's launches
+
+
+def test_fuzz_through_the_debug_build():
+    """The seeded random shapes of test_gpu_fuzz.py (T from 1, E up to 256, top-1
+    to top-8, both activations and storage types, capacity limits, threshold
+    gating, the k = 1 matmul) through the debug build, in a child process: every
+    case asserts MOE_OK, so no device bounds check may fire."""
+    env = dict(os.environ, MOE_LIBRARY="debug", PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_gpu_fuzz.py")],
+                       env=env, capture_output=True, text=True, timeout=1200, cwd=ROOT)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout
