@@ -74,7 +74,10 @@ typedef enum {
 typedef void* moe_stream_t;  /* a cudaStream_t; NULL = the legacy default stream */
 
 /* Bytes of workspace that every entry point below needs for these sizes
- * (the fused moe_forward needs the most; one size serves every call).     */
+ * (the fused moe_forward needs the most; one size serves every call).  For
+ * bf16 layers it includes 40 MiB of fp32 partial sums and 16 KiB of tickets
+ * with which the SwiGLU expert GEMM cuts its last partial wave of tiles in
+ * two along K (results deterministic; see moe_forward).                    */
 size_t moe_workspace_bytes(int T, int H, int F, int E, int top_k, moe_act act, moe_dtype dt);
 
 /* Router.  [P2] §2.1 (gates = softmax(x @ W_gate), top_k(gates, k=2)), §3.2.1
@@ -182,7 +185,13 @@ moe_status moe_unpermute_combine(const void* y, const float* topk_gate, const in
  * stream with no host synchronisation.  [P3] MoEOperator::Forward; [P5] ch.8
  * moe_router(x, router_weight, expert_weights, top_k, normalize_scores=True,
  * capacity_factor); [P4] §1 (fusing permute, matmul, softmax, experts, combine).
- * topk_idx_out [T,k] and expert_counts_out [E] (pre-drop) may be NULL.      */
+ * topk_idx_out [T,k] and expert_counts_out [E] (pre-drop) may be NULL.
+ * Results are the same bit for bit on every run of the same inputs on the
+ * same GPU model.  The SwiGLU GEMM may add the two K halves of its last
+ * partial wave of tiles in fp32 (which tiles depends on the expert counts and
+ * the SM count), so two layers whose routing differs may round a token's
+ * output differently in the last bit; the tolerance against exact arithmetic
+ * is unchanged.                                                            */
 moe_status moe_forward(const void* x, const void* w_gate, const float* gate_bias,
                        const void* w1, const void* w3, const void* w2,
                        int T, int H, int F, int E, int top_k, float capacity_factor,
